@@ -1,0 +1,206 @@
+"""Quantized block-sparse attention forward (EagleQBSA), step by step in fp64.
+
+Source: EagleQBSA article, "昇腾MindIE SD高性能量化稀疏联合注意力EagleQBSA,视频生成端到端加速1.6倍".
+
+* Section "EagleQBSA量化叠加稀疏方案设计" and Fig 2.1: Q and K are quantised to
+  INT8, symmetric and linear, one scale per 128-token block of the sequence axis;
+  V is quantised to FP8 E4M3 with one scale per channel (head-dim column) covering
+  the whole sequence; the attention probabilities P are rounded to FP8 before P·V.
+* Section "MindIE SD调用方式": the operator receives the INT8 query/key, the E4M3
+  value bytes, query_scale / key_scale / value_scale, a block_sparse_mask with
+  block_shape [128, 128], scale_value (the softmax scale, 128^-0.5 in the example)
+  and num_key_value_heads; the output is bf16.
+* Section "背景介绍": only the selected blocks of the attention map are computed.
+
+Readings where the article is silent (each also listed in the design notes):
+
+* Quantiser: a = max |x| over the block (or channel) in float32; scale s = a / 127
+  (INT8) or a / 448 (E4M3) in float32, and s = 1 when a = 0; INT8 codes are
+  rint_half_even(x / s) clamped to [-127, 127]; E4M3 codes are x / s rounded to
+  nearest even with saturation.  A tail block (S % 128 != 0) gets its own scale.
+* Shapes: query_scale [B, N_q, ceil(S_q/128)], key_scale [B, N_kv, ceil(S_kv/128)],
+  value_scale [B, N_kv, D]; block_sparse_mask uint8 [B, N_q, ceil(S_q/128),
+  ceil(S_kv/128)] with 1 = compute the block.
+* Score: s = t * s_q * s_k * scale, t the exact integer dot product of the INT8 rows.
+* Kept blocks are visited in ascending key order; the softmax runs online, one
+  128-key block per step: m_new = max(m, rowmax s); p = exp(s - m_new) held in
+  float32 (the precision in which the FP8 rounding decision is taken) and rounded to
+  E4M3 (nearest even); l = l * exp(m - m_new) + Σ p8 (the sum of the ROUNDED
+  weights); acc = acc * exp(m - m_new) + p8 · v8.
+* Output O[:, c] = acc[:, c] / l * v_scale[c]; softmax_max = final m; softmax_sum =
+  final l.  A row with no kept block returns O = 0, max = -inf, sum = 0.
+
+Parity pins (tests): the quantiser codes meet the rounding bound |x - q s| <= s/2 and
+hit ±127 at the block maximum; the E4M3 codec matches the OCP definition on every
+code and torch's float8_e4m3fn cast on finite inputs; with P rounding switched off the
+online recurrence equals the direct softmax over the kept keys; q = 0 gives p8 = 1,
+softmax_sum = 128 x kept blocks and O = the mean of the dequantised V; constant V
+returns V; a pure-Python loop version agrees on tiny inputs; masked-out blocks have
+no influence.  The article prints no quantisation error figure ("parity unpinned"
+for the article's own error level; only VBench scores are given, out of scope).
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+from .formats import bf16_to_f64, e4m3_encode, e4m3_decode
+
+BLK = 128
+
+
+# --------------------------------------------------------------------------------------
+# quantisers
+# --------------------------------------------------------------------------------------
+
+def _f32_values(x):
+    x = np.asarray(x)
+    if x.dtype == np.uint16:
+        return bf16_to_f64(x).astype(np.float32)
+    return x.astype(np.float32)
+
+
+def quantize_qk_per_block(x, block: int = BLK):
+    """x [B, N, S, D] (bf16 bits or float32) -> (int8 codes [B, N, S, D], float32 scales [B, N, nblk])."""
+    xf = _f32_values(x)
+    B, N, S, D = xf.shape
+    nblk = -(-S // block)
+    codes = np.zeros((B, N, S, D), dtype=np.int8)
+    scales = np.zeros((B, N, nblk), dtype=np.float32)
+    for kb in range(nblk):
+        r0, r1 = kb * block, min(S, (kb + 1) * block)
+        blk = xf[:, :, r0:r1, :]
+        a = np.abs(blk).max(axis=(2, 3)).astype(np.float32)
+        s = np.where(a == 0, np.float32(1.0), a / np.float32(127.0)).astype(np.float32)
+        q = np.rint(blk / s[:, :, None, None])
+        codes[:, :, r0:r1, :] = np.clip(q, -127, 127).astype(np.int8)
+        scales[:, :, kb] = s
+    return codes, scales
+
+
+def quantize_v_per_channel(v):
+    """v [B, N, S, D] (bf16 bits or float32) -> (E4M3 codes uint8 [B, N, S, D], float32 scales [B, N, D])."""
+    vf = _f32_values(v)
+    a = np.abs(vf).max(axis=2).astype(np.float32)
+    s = np.where(a == 0, np.float32(1.0), a / np.float32(448.0)).astype(np.float32)
+    codes = e4m3_encode((vf / s[:, :, None, :]).astype(np.float32))
+    return codes, s
+
+
+# --------------------------------------------------------------------------------------
+# the forward
+# --------------------------------------------------------------------------------------
+
+def _head_forward(q8, k8, qs, ks, v8f, vs, mask_rows, scale, skv, qbs, round_p=True):
+    """One (b, h): q8 [Sq, D] int8, k8 [Skv, D], v8f [Skv, D] decoded E4M3, per-block scales."""
+    D = v8f.shape[1]
+    outs, mxs, sms = [], [], []
+    for qb in qbs:
+        r0, r1 = qb * BLK, min(q8.shape[0], (qb + 1) * BLK)
+        rows = r1 - r0
+        m = np.full(rows, -np.inf)
+        l = np.zeros(rows)
+        acc = np.zeros((rows, D))
+        qi = q8[r0:r1].astype(np.int64)
+        for kb in np.nonzero(mask_rows[qb])[0]:
+            c0, c1 = kb * BLK, min(skv, (kb + 1) * BLK)
+            t = qi @ k8[c0:c1].astype(np.int64).T                     # exact integers
+            s = t.astype(np.float64) * (float(qs[qb]) * float(ks[kb]) * scale)
+            m_new = np.maximum(m, s.max(axis=1))
+            alpha = np.where(np.isfinite(m), np.exp(m - m_new), 0.0)
+            p = np.exp(s - m_new[:, None])
+            if round_p:
+                p = e4m3_decode(e4m3_encode(p.astype(np.float32)))
+            l = l * alpha + p.sum(axis=1)
+            acc = acc * alpha[:, None] + p @ v8f[c0:c1]
+            m = m_new
+        live = l > 0
+        o = np.where(live[:, None], acc / np.where(live, l, 1.0)[:, None], 0.0) * vs[None, :]
+        outs.append(o)
+        mxs.append(m)
+        sms.append(l)
+    return outs, mxs, sms
+
+
+def qbsa_forward(q8, k8, q_scale, k_scale, v8, v_scale, block_mask, scale: float,
+                 heads=None, q_blocks=None, round_p: bool = True):
+    """Oracle of the quantized block-sparse forward (BNSD).
+
+    q8 [B, Nq, Sq, D] int8; k8 [B, Nkv, Skv, D] int8; q_scale [B, Nq, ceil(Sq/128)];
+    k_scale [B, Nkv, ceil(Skv/128)]; v8 [B, Nkv, Skv, D] E4M3 codes (uint8);
+    v_scale [B, Nkv, D]; block_mask [B, Nq, ceil(Sq/128), ceil(Skv/128)] uint8, 1 = compute.
+
+    Returns (out [B, Nq, Sq, D], softmax_max [B, Nq, Sq], softmax_sum [B, Nq, Sq]) in
+    fp64.  ``heads`` / ``q_blocks`` restrict the work for sampled checks (other entries
+    NaN).  ``round_p=False`` skips the FP8 rounding of P (used only by a pin).
+    """
+    q8 = np.asarray(q8)
+    k8 = np.asarray(k8)
+    B, Nq, Sq, D = q8.shape
+    Nkv, Skv = k8.shape[1], k8.shape[2]
+    group = Nq // Nkv
+    nqb = -(-Sq // BLK)
+    out = np.full((B, Nq, Sq, D), np.nan)
+    smax = np.full((B, Nq, Sq), np.nan)
+    ssum = np.full((B, Nq, Sq), np.nan)
+    sel = heads if heads is not None else [(b, h) for b in range(B) for h in range(Nq)]
+    qbs = list(range(nqb)) if q_blocks is None else list(q_blocks)
+    v8f_cache = {}
+    for b, h in sel:
+        g = h // group
+        if (b, g) not in v8f_cache:
+            v8f_cache[(b, g)] = e4m3_decode(v8[b, g])
+        o, mx, sm = _head_forward(q8[b, h], k8[b, g], q_scale[b, h], k_scale[b, g],
+                                  v8f_cache[(b, g)], np.asarray(v_scale[b, g], dtype=np.float64),
+                                  block_mask[b, h], scale, Skv, qbs, round_p)
+        for qb, oo, mm, ss in zip(qbs, o, mx, sm):
+            r0, r1 = qb * BLK, min(Sq, (qb + 1) * BLK)
+            out[b, h, r0:r1] = oo
+            smax[b, h, r0:r1] = mm
+            ssum[b, h, r0:r1] = ss
+    return out, smax, ssum
+
+
+def qbsa_forward_loops(q8, k8, q_scale, k_scale, v8, v_scale, block_mask, scale: float):
+    """The same forward with explicit Python loops over rows, blocks and keys (tiny inputs)."""
+    import math
+    q8 = np.asarray(q8)
+    k8 = np.asarray(k8)
+    B, Nq, Sq, D = q8.shape
+    Nkv, Skv = k8.shape[1], k8.shape[2]
+    group = Nq // Nkv
+    out = np.zeros((B, Nq, Sq, D))
+    smax = np.full((B, Nq, Sq), -np.inf)
+    ssum = np.zeros((B, Nq, Sq))
+    for b in range(B):
+        for h in range(Nq):
+            g = h // group
+            for i in range(Sq):
+                qb = i // BLK
+                m, l = -math.inf, 0.0
+                acc = [0.0] * D
+                for kb in range(block_mask.shape[3]):
+                    if not block_mask[b, h, qb, kb]:
+                        continue
+                    cols = range(kb * BLK, min(Skv, (kb + 1) * BLK))
+                    s = []
+                    for j in cols:
+                        t = sum(int(q8[b, h, i, c]) * int(k8[b, g, j, c]) for c in range(D))
+                        s.append(t * (float(q_scale[b, h, qb]) * float(k_scale[b, g, kb]) * scale))
+                    m_new = max(m, max(s))
+                    alpha = math.exp(m - m_new) if m != -math.inf else 0.0
+                    l *= alpha
+                    acc = [a * alpha for a in acc]
+                    for j, sj in zip(cols, s):
+                        p = float(e4m3_decode(e4m3_encode(np.float32(math.exp(sj - m_new)))))
+                        l += p
+                        vrow = e4m3_decode(v8[b, g, j])
+                        for c in range(D):
+                            acc[c] += p * vrow[c]
+                    m = m_new
+                if l > 0:
+                    for c in range(D):
+                        out[b, h, i, c] = acc[c] / l * float(v_scale[b, g, c])
+                smax[b, h, i] = m
+                ssum[b, h, i] = l
+    return out, smax, ssum
