@@ -1,0 +1,431 @@
+#!/usr/bin/env python
+"""Throughput of the fused attention forward on B200, one JSON line on rank 0.
+
+Default workload (one step = one qbsa_fwd call): quantized block-sparse attention,
+B=1, N=40, S=65536, D=128, INT8 Q/K per 128-token block, E4M3 V per channel, 128x128
+block mask keeping 10% of the blocks per (head, query block) with the diagonal kept.
+The dense bf16 video workload (attn_fwd, B=1, N=40, S=61440, D=128) is timed beside
+it and reported under "extra".  ``--sweep`` adds the S sweep 8K..128K at keep 0.1 and
+0.5 (and dense) as extra lines.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU (torchrun, one rank per GPU): every rank runs the same per-GPU workload
+(the heads are independent; no collective on the data path) and ``value`` is the
+total work of all ranks divided by the max over ranks of the timed span ("weak").
+``--impl reference`` times the CPU oracle on a bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd TFLOPS (B=1,N=40,D=128) and % of B200 tensor peak vs S"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FP8_OVER_BF16 = 2.0  # nominal dense ratio (4.5 vs 2.25 PFLOP/s), applied to the measured bf16 peak
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--seq", type=int, default=65536)
+    p.add_argument("--keep", type=float, default=0.1)
+    p.add_argument("--sweep", action="store_true")
+    p.add_argument("--no-dense", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu", action="store_true")
+    return p.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------------------------
+# clocks during the timed region
+# ----------------------------------------------------------------------------------
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                                         stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx = max(mx, float(parts[2]))
+                except ValueError:
+                    continue
+                for nm, val in zip(names, parts[5:9]):
+                    if val.lower() == "active":
+                        reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------------
+# workloads
+# ----------------------------------------------------------------------------------
+
+def qbsa_inputs(S: int, keep: float, device):
+    """Device-resident quantized inputs of the block-sparse workload (B=1, N=40, D=128)."""
+    import numpy as np
+    import torch
+    import quantized_block_sparse_attn_b200 as qb
+    from workloads import CONFIGS, block_keep_mask, device_blocky_qk_bf16, device_iid_normal_bf16
+    c = CONFIGS["qbsa"]
+    N, D, seed = c["Nq"], c["D"], c["seed"]
+    q = device_blocky_qk_bf16(seed, "q", 1, N, S, D, device)
+    k = device_blocky_qk_bf16(seed, "k", 1, N, S, D, device)
+    v = device_iid_normal_bf16(seed, 2, (1, N, S, D), device)
+    q8, qs = qb.quantize_qk(q)
+    k8, ks = qb.quantize_qk(k)
+    v8, vs = qb.quantize_v(v)
+    torch.cuda.synchronize(device)
+    del q, k, v
+    nb = -(-S // 128)
+    bm_np = block_keep_mask(seed, 1, N, nb, nb, keep)
+    bm = torch.from_numpy(bm_np).to(device)
+    kept = int(bm_np.sum())
+    return dict(q8=q8, qs=qs, k8=k8, ks=ks, v8=v8, vs=vs, bm=bm, bm_np=bm_np, kept=kept, N=N, D=D, S=S,
+                scale=c["scale"], seed=seed)
+
+
+def qbsa_work(inp):
+    """Executed FLOPs (kept blocks), dense-equivalent FLOPs and algorithmic bytes of one call."""
+    N, S, D, kept = inp["N"], inp["S"], inp["D"], inp["kept"]
+    executed = 4.0 * D * 128 * 128 * kept
+    dense_eq = 4.0 * D * S * S * N
+    nb = -(-S // 128)
+    bytes_ = 3 * N * S * D + 2 * N * S * D + N * nb * nb + 4 * (2 * N * nb + N * D)
+    return executed, dense_eq, bytes_
+
+
+def time_steps(fn, steps: int, warmup: int, stream, dist=None, sampler=None):
+    """Run fn warmup times, then time exactly `steps` calls with CUDA events on `stream`."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    evs[0].record(stream)
+    for i in range(steps):
+        fn()
+        evs[i + 1].record(stream)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = sampler.stop() if sampler else None
+    per = [evs[i].elapsed_time(evs[i + 1]) for i in range(steps)]
+    total = evs[0].elapsed_time(evs[-1])
+    return total, per, clocks
+
+
+def max_over_ranks(x: float, dist):
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def cpu_oracle_sample(inp_host, n_qblocks: int):
+    """Time the oracle (as it stands) on n_qblocks query blocks of head 0.  Returns (TFLOP/s, s, desc)."""
+    import numpy as np
+    from oracle import quant
+    from workloads import sample_rows
+    S, D = inp_host["S"], inp_host["D"]
+    qbs = sample_rows(inp_host["seed"], S, n_qblocks)
+    bm = inp_host["bm_np"][:, :1]
+    t0 = time.perf_counter()
+    quant.qbsa_forward(inp_host["q8"], inp_host["k8"], inp_host["qs"], inp_host["ks"], inp_host["v8"],
+                       inp_host["vs"], bm, inp_host["scale"], q_blocks=qbs)
+    dt = time.perf_counter() - t0
+    kept = int(bm[0, 0, qbs].sum())
+    flops = 4.0 * D * 128 * 128 * kept
+    return flops / dt / 1e12, dt, f"head 0, {len(qbs)} query blocks ({kept} kept 128x128 blocks) of S={S}"
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        n = max((i.get("num_threads", 1) for i in info), default=1)
+        return int(n)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def host_head0(inp):
+    """Host copies of head 0's quantized inputs (for the CPU oracle sample)."""
+    return dict(q8=inp["q8"][:, :1].cpu().numpy(), k8=inp["k8"][:, :1].cpu().numpy(),
+                qs=inp["qs"][:, :1].cpu().numpy(), ks=inp["ks"][:, :1].cpu().numpy(),
+                v8=inp["v8"][:, :1].cpu().numpy(), vs=inp["vs"][:, :1].cpu().numpy(), bm_np=inp["bm_np"],
+                S=inp["S"], D=inp["D"], scale=inp["scale"], seed=inp["seed"])
+
+
+# ----------------------------------------------------------------------------------
+# arms
+# ----------------------------------------------------------------------------------
+
+def run_reference(args):
+    """CPU oracle arm: each step is one query block of head 0 of the same workload."""
+    import numpy as np
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from oracle import quant
+    from workloads import CONFIGS, block_keep_mask, blocky_qk_bf16, iid_normal_bf16, sample_rows
+    c = CONFIGS["qbsa"]
+    S, D, seed = args.seq, c["D"], c["seed"]
+    # head 0 only, generated on the host; quantised by the oracle's own quantiser
+    q = blocky_qk_bf16(seed, "q", 1, 1, S, D)
+    k = blocky_qk_bf16(seed, "k", 1, 1, S, D)
+    v = iid_normal_bf16(seed, 2, 1, 1, S, D)
+    q8, qs = quant.quantize_qk_per_block(q)
+    k8, ks = quant.quantize_qk_per_block(k)
+    v8, vs = quant.quantize_v_per_channel(v)
+    nb = S // 128
+    bm = block_keep_mask(seed, 1, 1, nb, nb, args.keep)
+    qbs = sample_rows(seed, S, args.steps + args.warmup)
+    while len(qbs) < args.steps + args.warmup:
+        qbs = qbs + qbs
+    times, flops = [], []
+    for i in range(args.warmup + args.steps):
+        qb_ = qbs[i]
+        t0 = time.perf_counter()
+        quant.qbsa_forward(q8, k8, qs, ks, v8, vs, bm, c["scale"], q_blocks=[qb_])
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            times.append(dt)
+            flops.append(4.0 * D * 128 * 128 * int(bm[0, 0, qb_].sum()))
+    tot = sum(times)
+    value = sum(flops) / tot / 1e12
+    cores = blas_threads()
+    sample = f"one query block of head 0 per step (S={S}, keep={args.keep}), {args.steps} steps"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "i8+e4m3 (emulated in f64)",
+            "data": "synthetic",
+            "config": {"workload": f"qbsa_fwd B=1 N=40 S={S} D=128 keep={args.keep}", "global_batch": 1,
+                       "seq_len": S, "parallelism": "cpu oracle, rank 0 only"},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+
+
+def run_ours(args):
+    import torch
+    import quantized_block_sparse_attn_b200 as qb
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as tdist
+        torch.cuda.set_device(local)
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                 device_id=torch.device("cuda", local))
+        dist = tdist
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    stream = torch.cuda.current_stream(device)
+    peaks, peak_src = load_peaks()
+    fp8_peak = peaks["bf16_tflops"] * FP8_OVER_BF16
+    bf16_peak = peaks["bf16_tflops"]
+
+    # ---------------------------------------------------------------- main: qbsa_fwd
+    inp = qbsa_inputs(args.seq, args.keep, device)
+    executed, dense_eq, alg_bytes = qbsa_work(inp)
+    out = torch.empty((1, inp["N"], inp["S"], inp["D"]), dtype=torch.bfloat16, device=device)
+
+    def step():
+        qb.qbsa_fwd(inp["q8"], inp["k8"], inp["qs"], inp["ks"], inp["v8"], inp["vs"], inp["bm"], inp["scale"],
+                    out=out, return_stats=False)
+
+    sampler = ClockSampler(local)
+    total_ms, per_ms, clocks = time_steps(step, args.steps, args.warmup, stream, dist, sampler)
+    qb.check(device)
+    total_ms = max_over_ranks(total_ms, dist)
+    ms_step = total_ms / args.steps
+    value = world * executed * args.steps / (total_ms / 1e3) / 1e12
+    launch_ms = sum(per_ms) / len(per_ms)
+    achieved = executed / (launch_ms / 1e3) / 1e12
+
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "i8xi8->s32, e4m3xe4m3->f32, bf16 out", "data": "synthetic",
+            "config": {"workload": f"qbsa_fwd B=1 N=40 S={args.seq} D=128 keep={args.keep} (per GPU)",
+                       "global_batch": world, "seq_len": args.seq, "parallelism": f"dp{world} (heads independent)",
+                       "l2": f"inputs {3 * inp['N'] * inp['S'] * inp['D'] / 1e9:.2f} GB > 126 MB L2, no flush",
+                       "dense_equivalent_tflops": world * dense_eq * args.steps / (total_ms / 1e3) / 1e12,
+                       "pct_of_fp8_int8_peak": 100.0 * achieved / fp8_peak},
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": fp8_peak, "unit": "TFLOP/s",
+                         "frac": achieved / fp8_peak, "traffic": None,
+                         "peak_source": f"{peak_src} bf16 burst {bf16_peak} x {FP8_OVER_BF16} (nominal fp8/int8:bf16)",
+                         "kernel": "attn_qbsa_kernel", "algorithmic_bytes": alg_bytes,
+                         "hbm_gbs_algorithmic": alg_bytes / (launch_ms / 1e3) / 1e9},
+            "gpu_launches": args.steps, "clocks": clocks}
+
+    # ---------------------------------------------------------------- e2e through the public API, host buffers
+    if not args.no_e2e:
+        host = {k: inp[k].cpu().pin_memory() for k in ("q8", "qs", "k8", "ks", "v8", "vs", "bm")}
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = out.numel() * out.element_size()
+        e2e_steps = max(2, min(5, args.steps))
+
+        def e2e_step():
+            res = qb.qbsa_fwd(host["q8"], host["k8"], host["qs"], host["ks"], host["v8"], host["vs"], host["bm"],
+                              inp["scale"], return_stats=False, device=device)
+            return res[0]
+
+        e2e_step()
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        t0 = time.perf_counter()
+        for _ in range(e2e_steps):
+            e2e_step()
+        torch.cuda.synchronize()
+        e2e_s = max_over_ranks((time.perf_counter() - t0) / e2e_steps, dist)
+        line["e2e"] = {"value": world * executed / e2e_s / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                       "d2h_bytes_per_step": d2h, "ms_per_step": 1e3 * e2e_s,
+                       "note": "host pinned int8/e4m3/fp32 inputs copied in, bf16 output copied out, every step"}
+
+    # ---------------------------------------------------------------- CPU oracle sample (rank 0, N=1)
+    if rank == 0 and world == 1 and not args.no_cpu:
+        tf, secs, desc = cpu_oracle_sample(host_head0(inp), n_qblocks=24)
+        line["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+                                "sample": desc + f", {secs:.1f} s"}
+
+    extra = {}
+    del inp
+    torch.cuda.empty_cache()
+    # ---------------------------------------------------------------- dense bf16 video workload
+    if not args.no_dense:
+        extra["dense_video"] = dense_line(device, stream, 61440, max(2, args.warmup), 3, bf16_peak, dist)
+    if args.sweep:
+        for S in (8192, 16384, 32768, 65536, 131072):
+            for keep in (0.1, 0.5):
+                extra[f"qbsa_S{S}_keep{keep}"] = qbsa_line(device, stream, S, keep, fp8_peak)
+            extra[f"dense_S{S}"] = dense_line(device, stream, S, 2, 3, bf16_peak, None)
+    if extra:
+        line["extra"] = extra
+    if dist is not None:
+        dist.barrier()
+    if rank == 0:
+        print(json.dumps(line))
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+def qbsa_line(device, stream, S, keep, fp8_peak):
+    import torch
+    import quantized_block_sparse_attn_b200 as qb
+    inp = qbsa_inputs(S, keep, device)
+    executed, dense_eq, _ = qbsa_work(inp)
+    out = torch.empty((1, inp["N"], S, inp["D"]), dtype=torch.bfloat16, device=device)
+
+    def step():
+        qb.qbsa_fwd(inp["q8"], inp["k8"], inp["qs"], inp["ks"], inp["v8"], inp["vs"], inp["bm"], inp["scale"],
+                    out=out, return_stats=False)
+
+    total, per, _ = time_steps(step, 5, 2, stream)
+    ms = total / 5
+    del inp
+    torch.cuda.empty_cache()
+    return {"S": S, "keep": keep, "ms": ms, "executed_tflops": executed / ms / 1e9,
+            "dense_equivalent_tflops": dense_eq / ms / 1e9, "pct_of_fp8_peak": 100 * executed / ms / 1e9 / fp8_peak}
+
+
+def dense_line(device, stream, S, warmup, steps, bf16_peak, dist):
+    import torch
+    import quantized_block_sparse_attn_b200 as qb
+    from workloads import CONFIGS, device_blocky_qk_bf16, device_iid_normal_bf16
+    c = CONFIGS["video"]
+    N, D, seed = c["Nq"], c["D"], c["seed"]
+    q = device_blocky_qk_bf16(seed, "q", 1, N, S, D, device)
+    k = device_blocky_qk_bf16(seed, "k", 1, N, S, D, device)
+    v = device_iid_normal_bf16(seed, 2, (1, N, S, D), device)
+    out = torch.empty_like(q)
+
+    def step():
+        qb.attn_fwd(q, k, v, N, "BNSD", scale=c["scale"], out=out, return_stats=False)
+
+    total, per, clocks = time_steps(step, steps, warmup, stream, dist)
+    qb.check(device)
+    ms = max_over_ranks(total / steps, dist)
+    flops = 4.0 * D * S * S * N
+    del q, k, v, out
+    torch.cuda.empty_cache()
+    return {"workload": f"attn_fwd bf16 B=1 N=40 S={S} D=128 no mask", "ms": ms, "tflops": flops / ms / 1e9,
+            "pct_of_bf16_peak": 100 * flops / ms / 1e9 / bf16_peak, "kernel": "attn_dense_kernel<128>"}
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

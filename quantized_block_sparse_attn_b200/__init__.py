@@ -1,0 +1,19 @@
+"""B200 (sm_100a) fused attention forward: dense bf16 and quantized block-sparse (EagleQBSA).
+
+The compute path is libqbsa.so (hand-written tcgen05 / TMA / TMEM kernels behind a C
+ABI, declared in include/qbsa.h); this package is its thin ctypes binding.
+"""
+
+from ._binding import (  # noqa: F401
+    INF_TOKENS,
+    LIB_PATH,
+    QbsaError,
+    attn_fwd,
+    attn_tile_schedule,
+    block_lists,
+    check,
+    lib,
+    qbsa_fwd,
+    quantize_qk,
+    quantize_v,
+)

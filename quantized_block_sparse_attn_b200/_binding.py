@@ -1,0 +1,219 @@
+"""ctypes binding of libqbsa.so: argument marshalling only.
+
+Every numeric step runs in the library's CUDA kernels.  PyTorch supplies device
+memory and the current stream.  There is no CPU fallback: if the library has not
+been built (``python -m quantized_block_sparse_attn_b200.build``) or the CUDA path
+cannot run, calls raise.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+_LIB = None
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libqbsa.so")
+
+STATUS = {0: "QBSA_OK", 1: "QBSA_ERR_INVALID", 2: "QBSA_ERR_UNSUPPORTED", 3: "QBSA_ERR_CUDA", 4: "QBSA_ERR_TIMEOUT"}
+LAYOUTS = {"BNSD": 0, "BSND": 1, "TND": 2}
+MASK_SHAPES = {None: 0, "SS": 1, "B1SS": 2, "BNSS": 3}
+INF_TOKENS = 2147483647
+
+# exported symbol -> (restype, argtypes)
+_P, _I, _I64, _F = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float
+SIGNATURES = {
+    "attn_fwd": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _I, _P, _I, _F, _F, _I, _I64, _I64,
+                      _P, _P, _P, _P, _P, _P]),
+    "qbsa_fwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P]),
+    "qbsa_quantize_qk": (_I, [_P, _I, _I, _I, _I, _P, _P, _P]),
+    "qbsa_quantize_v": (_I, [_P, _I, _I, _I, _I, _P, _P, _P]),
+    "attn_tile_schedule": (_I, [_I64, _I64, _I, _I64, _I64, _P, _P, _P, _P, _I64]),
+    "qbsa_block_lists": (_I, [_P, _I64, _I, _P, _P, _P]),
+    "qbsa_check": (_I, [_P]),
+    "qbsa_last_error": (ctypes.c_char_p, []),
+    "qbsa_version": (_I, []),
+}
+
+
+class QbsaError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS.get(status, status)}: {message}")
+        self.status = status
+
+
+def lib():
+    """Load libqbsa.so (once).  Raises if it has not been built."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m quantized_block_sparse_attn_b200.build`")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(handle, name)
+            fn.restype = res
+            fn.argtypes = args
+        _LIB = handle
+    return _LIB
+
+
+def _ck(status: int):
+    if status != 0:
+        raise QbsaError(status, lib().qbsa_last_error().decode("utf-8", "replace"))
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device):
+    import torch
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _on_cuda(tensors, device):
+    """Host tensors are copied to the device (pinned, asynchronous); device tensors pass through."""
+    import torch
+    out = []
+    for t in tensors:
+        if t is None or t.is_cuda:
+            out.append(t)
+        else:
+            src = t if t.is_pinned() else t.pin_memory()
+            out.append(src.to(device, non_blocking=True))
+    return out
+
+
+def attn_fwd(q, k, v, head_num: int, input_layout: str = "BNSD", *, atten_mask=None, mask_shape=None, pse=None,
+             scale: float = 1.0, keep_prob: float = 1.0, sparse_mode: int = 0, pre_tokens: int = INF_TOKENS,
+             next_tokens: int = INF_TOKENS, actual_seq_qlen=None, actual_seq_kvlen=None, out=None,
+             softmax_max=None, softmax_sum=None, return_stats: bool = True, device=None):
+    """Dense fused attention forward (bf16).  Returns (attention_out, softmax_max, softmax_sum).
+
+    Tensors may live on the GPU or on the host; host inputs are copied to ``device``
+    (default cuda:0) and the results are copied back to the host.
+    """
+    import torch
+    host = not q.is_cuda
+    dev = torch.device(device or (q.device if q.is_cuda else "cuda:0"))
+    q, k, v, atten_mask, pse = _on_cuda([q, k, v, atten_mask, pse], dev)
+    for t in (q, k, v):
+        if t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous bfloat16 tensors")
+    lay = LAYOUTS[input_layout]
+    if input_layout == "BNSD":
+        B, Nq, Sq, D = q.shape
+        Nkv, Skv = k.shape[1], k.shape[2]
+    elif input_layout == "BSND":
+        B, Sq, Nq, D = q.shape
+        Skv, Nkv = k.shape[1], k.shape[2]
+    else:
+        Sq, Nq, D = q.shape
+        Skv, Nkv = k.shape[0], k.shape[1]
+        B = len(actual_seq_qlen)
+    cq = ck = None
+    if input_layout == "TND":
+        cq = np.ascontiguousarray(np.asarray(actual_seq_qlen, dtype=np.int64))
+        ck = np.ascontiguousarray(np.asarray(actual_seq_kvlen, dtype=np.int64))
+    if atten_mask is not None:
+        if atten_mask.dtype == torch.bool:
+            atten_mask = atten_mask.to(torch.uint8)
+        atten_mask = atten_mask.contiguous()
+        if mask_shape is None:
+            mask_shape = {2: "SS", 4: "BNSS" if atten_mask.shape[1] == Nq and Nq > 1 else "B1SS"}[atten_mask.dim()]
+    pse_bcast = 0
+    if pse is not None:
+        pse = pse.contiguous()
+        pse_bcast = int(pse.shape[0] == 1 and B > 1)
+    if out is None:
+        out = torch.empty_like(q)
+    if return_stats:
+        sshape = (Nq, Sq) if input_layout == "TND" else (B, Nq, Sq)
+        if softmax_max is None:
+            softmax_max = torch.empty(sshape, dtype=torch.float32, device=dev)
+        if softmax_sum is None:
+            softmax_sum = torch.empty(sshape, dtype=torch.float32, device=dev)
+    L = lib()
+    _ck(L.attn_fwd(_ptr(q), _ptr(k), _ptr(v), B, Nq, Nkv, Sq, Skv, D, head_num, lay, _ptr(atten_mask),
+                   MASK_SHAPES[mask_shape], _ptr(pse), pse_bcast, scale, keep_prob, sparse_mode, pre_tokens,
+                   next_tokens, None if cq is None else cq.ctypes.data_as(ctypes.c_void_p),
+                   None if ck is None else ck.ctypes.data_as(ctypes.c_void_p), _ptr(out), _ptr(softmax_max),
+                   _ptr(softmax_sum), _stream(dev)))
+    if host:
+        return tuple(None if t is None else t.cpu() for t in (out, softmax_max, softmax_sum))
+    return out, softmax_max, softmax_sum
+
+
+def qbsa_fwd(q_i8, k_i8, q_scale, k_scale, v_fp8, v_scale, block_mask, scale: float, *, out=None,
+             softmax_max=None, softmax_sum=None, return_stats: bool = True, device=None):
+    """Quantized block-sparse attention forward (BNSD, D = 128).  Returns (out, max, sum)."""
+    import torch
+    host = not q_i8.is_cuda
+    dev = torch.device(device or (q_i8.device if q_i8.is_cuda else "cuda:0"))
+    q_i8, k_i8, q_scale, k_scale, v_fp8, v_scale, block_mask = _on_cuda(
+        [q_i8, k_i8, q_scale, k_scale, v_fp8, v_scale, block_mask], dev)
+    B, Nq, Sq, D = q_i8.shape
+    Nkv, Skv = k_i8.shape[1], k_i8.shape[2]
+    if out is None:
+        out = torch.empty((B, Nq, Sq, D), dtype=torch.bfloat16, device=dev)
+    if return_stats:
+        if softmax_max is None:
+            softmax_max = torch.empty((B, Nq, Sq), dtype=torch.float32, device=dev)
+        if softmax_sum is None:
+            softmax_sum = torch.empty((B, Nq, Sq), dtype=torch.float32, device=dev)
+    L = lib()
+    _ck(L.qbsa_fwd(_ptr(q_i8), _ptr(k_i8), _ptr(q_scale), _ptr(k_scale), _ptr(v_fp8), _ptr(v_scale),
+                   _ptr(block_mask), B, Nq, Nkv, Sq, Skv, D, scale, _ptr(out), _ptr(softmax_max),
+                   _ptr(softmax_sum), _stream(dev)))
+    if host:
+        return tuple(None if t is None else t.cpu() for t in (out, softmax_max, softmax_sum))
+    return out, softmax_max, softmax_sum
+
+
+def quantize_qk(x):
+    """Per-128-block INT8 quantisation of a BNSD bf16 device tensor -> (codes int8, scales fp32)."""
+    import torch
+    B, N, S, D = x.shape
+    codes = torch.empty((B, N, S, D), dtype=torch.int8, device=x.device)
+    scales = torch.empty((B, N, -(-S // 128)), dtype=torch.float32, device=x.device)
+    _ck(lib().qbsa_quantize_qk(_ptr(x), B, N, S, D, _ptr(codes), _ptr(scales), _stream(x.device)))
+    return codes, scales
+
+
+def quantize_v(v):
+    """Per-channel E4M3 quantisation of a BNSD bf16 device tensor -> (codes uint8, scales fp32)."""
+    import torch
+    B, N, S, D = v.shape
+    codes = torch.empty((B, N, S, D), dtype=torch.uint8, device=v.device)
+    scales = torch.empty((B, N, D), dtype=torch.float32, device=v.device)
+    _ck(lib().qbsa_quantize_v(_ptr(v), B, N, S, D, _ptr(codes), _ptr(scales), _stream(v.device)))
+    return codes, scales
+
+
+def attn_tile_schedule(sq: int, skv: int, sparse_mode: int = 0, pre_tokens: int = INF_TOKENS,
+                       next_tokens: int = INF_TOKENS):
+    """Host-only: per query tile, (kt_begin, kt_end, full_begin, full_end) arrays."""
+    n = -(-sq // 128)
+    arrs = [np.zeros(n, dtype=np.int32) for _ in range(4)]
+    _ck(lib().attn_tile_schedule(sq, skv, sparse_mode, pre_tokens, next_tokens,
+                                 *[a.ctypes.data_as(ctypes.c_void_p) for a in arrs], n))
+    return tuple(arrs)
+
+
+def block_lists(block_mask_rows):
+    """Device mask compaction hook: (rows, n_kb) uint8 device tensor -> (lists int32, counts int32)."""
+    import torch
+    rows, n_kb = block_mask_rows.shape
+    lists = torch.empty((rows, n_kb), dtype=torch.int32, device=block_mask_rows.device)
+    counts = torch.empty((rows,), dtype=torch.int32, device=block_mask_rows.device)
+    _ck(lib().qbsa_block_lists(_ptr(block_mask_rows.contiguous()), rows, n_kb, _ptr(lists), _ptr(counts),
+                               _stream(block_mask_rows.device)))
+    return lists, counts
+
+
+def check(device=None):
+    """Synchronise the current stream and raise if a kernel reported a device-side timeout."""
+    import torch
+    _ck(lib().qbsa_check(_stream(torch.device(device or "cuda:0"))))

@@ -1,0 +1,427 @@
+// Dense bf16 fused attention forward for sm_100a.
+//
+// Computes Softmax(Mask(Q·Kᵀ·scale + pse))·V (npu_fusion_attention guide,
+// "昇腾 NPU 融合注意力算子详解与迁移指南", §2 算子数学原理) one 128-row query tile per
+// CTA, streaming 128-row K/V tiles with an online softmax so that the score matrix
+// never reaches global memory (§2, the tiling remark).  Masks follow §4.2/§4.3,
+// varlen TND follows §4.3, GQA follows §7, and the outputs are attention_out,
+// softmax_max and softmax_sum (§5).
+//
+// CTA = 6 warps:
+//   warp 0      TMA producer: Q once, then K/V tiles into a 2-stage ring each.
+//   warp 1      TMEM owner + MMA issuer (one thread): S = Q Kᵀ (kind::f16, SS) into a
+//               double-buffered f32 TMEM tile, then O += P V (kind::f16, A = P from
+//               TMEM, B = V from shared memory, MN-major).
+//   warps 2..5  softmax: thread t owns query row 32*(warp%4)+lane (its TMEM lane),
+//               loads its S row, masks, keeps the running max, rescales O in TMEM
+//               only when the max grew by more than 2^8 (the output is unchanged
+//               by the lagging reference; the statistics are corrected at the end),
+//               writes P as bf16 into TMEM and finally normalises O and stores it.
+// TMEM columns: S0 [0,128) S1 [128,256) O [256,256+D) P0 [384,448) P1 [448,512).
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "ptx_sm100.cuh"
+#include "schedule.cuh"
+
+namespace qbsa {
+
+constexpr int kMaxSeqs = 128;  // TND sequences per call (kernel-parameter tables, < 4 KB of params)
+
+struct DenseParams {
+  CUtensorMap tm_q;  // 4-D {D, rows, heads, batch}, box {64, 128, 1, 1}, bf16, SW128
+  CUtensorMap tm_k;
+  CUtensorMap tm_v;
+  __nv_bfloat16* out;
+  float* softmax_max;
+  float* softmax_sum;
+  const uint8_t* atten_mask;   // 1 = masked; nullptr if none
+  const __nv_bfloat16* pse;    // nullptr if none
+  int64_t o_row_stride, o_head_stride, o_batch_stride;  // elements
+  int64_t m_row_stride, m_head_stride, m_batch_stride;  // atten_mask strides (elements)
+  int64_t p_row_stride, p_head_stride, p_batch_stride;  // pse strides (elements)
+  int64_t stat_head_stride, stat_batch_stride;          // stats strides (elements)
+  int64_t pre_tokens, next_tokens;
+  int B, Nq, Nkv, Sq, Skv, group;
+  int sparse_mode;
+  int tnd;       // 1: varlen TND
+  int n_qtiles;  // BNSD/BSND: ceil(Sq/128)
+  float scale;
+  // TND tables (sequences in processing order)
+  int n_seq;
+  int seq_q_start[kMaxSeqs];
+  int seq_q_len[kMaxSeqs];
+  int seq_kv_start[kMaxSeqs];
+  int seq_kv_len[kMaxSeqs];
+  int seq_tile_start[kMaxSeqs + 1];
+};
+
+template <int D>
+struct DenseCfg {
+  static constexpr int kStages = 2;
+  static constexpr int kTileBytes = kTile * D * 2;  // one 128 x D bf16 tile
+  static constexpr int kSubBytes = kTile * 128;     // one 128-row x 128-byte swizzle column
+  static constexpr int kQOff = 0;
+  static constexpr int kKOff = kQOff + kTileBytes;
+  static constexpr int kVOff = kKOff + kStages * kTileBytes;
+  static constexpr int kBarOff = kVOff + kStages * kTileBytes;
+  // barriers
+  static constexpr int kBarQFull = 0;
+  static constexpr int kBarKFull = 1;
+  static constexpr int kBarKEmpty = kBarKFull + kStages;
+  static constexpr int kBarVFull = kBarKEmpty + kStages;
+  static constexpr int kBarVEmpty = kBarVFull + kStages;
+  static constexpr int kBarSFull = kBarVEmpty + kStages;  // 2
+  static constexpr int kBarSFree = kBarSFull + 2;         // 2
+  static constexpr int kBarPFull = kBarSFree + 2;         // 2
+  static constexpr int kBarPVDone = kBarPFull + 2;        // 1
+  static constexpr int kNumBars = kBarPVDone + 1;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  // + alignment slack; at least 120 KB so that one CTA holds an SM (and its 512 TMEM columns)
+  static constexpr int kSmemUsed = kMiscOff + 16 + 1024;
+  static constexpr int kSmemBytes = kSmemUsed > 120 * 1024 ? kSmemUsed : 120 * 1024;
+  // TMEM columns
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256, kColP0 = 384, kColP1 = 448;
+  static constexpr int kThreads = 192;
+};
+
+struct DenseWork {
+  int b, h, qt;
+  int64_t q_row0;   // tensor-map row coordinate of query row 0 of the tile's sequence
+  int64_t kv_row0;  // tensor-map row coordinate of key row 0 of the sequence
+  int coord_b;      // tensor-map batch coordinate
+  int64_t sq, skv;  // sequence lengths
+  int64_t tok0;     // TND: first token of the sequence (stats / output addressing)
+};
+
+__device__ __forceinline__ DenseWork dense_work(const DenseParams& p) {
+  DenseWork w;
+  // 1-D grid: heads fastest, so the first wave holds the heaviest tile of every head
+  w.h = static_cast<int>(blockIdx.x % p.Nq);
+  const int r = static_cast<int>(blockIdx.x / p.Nq);
+  if (!p.tnd) {
+    const int rank = r / p.B;
+    w.b = r % p.B;
+    w.qt = p.n_qtiles - 1 - rank;  // heaviest (causal) tiles first
+    w.q_row0 = 0;
+    w.kv_row0 = 0;
+    w.coord_b = w.b;
+    w.sq = p.Sq;
+    w.skv = p.Skv;
+    w.tok0 = 0;
+  } else {
+    int lo = 0, hi = p.n_seq - 1;
+    while (lo < hi) {  // last i with seq_tile_start[i] <= r
+      const int mid = (lo + hi + 1) >> 1;
+      if (p.seq_tile_start[mid] <= r) lo = mid; else hi = mid - 1;
+    }
+    const int ntile = p.seq_tile_start[lo + 1] - p.seq_tile_start[lo];
+    w.b = lo;  // index in processing order (tables are already permuted)
+    w.qt = ntile - 1 - (r - p.seq_tile_start[lo]);
+    w.q_row0 = p.seq_q_start[lo];
+    w.kv_row0 = p.seq_kv_start[lo];
+    w.coord_b = 0;
+    w.sq = p.seq_q_len[lo];
+    w.skv = p.seq_kv_len[lo];
+    w.tok0 = p.seq_q_start[lo];
+  }
+  return w;
+}
+
+template <int D>
+__global__ void __launch_bounds__(192, 1) attn_dense_kernel(const __grid_constant__ DenseParams p) {
+  using C = DenseCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_base = smem_u32(smem_raw);
+  const uint32_t base = (raw_base + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - raw_base);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t bar0 = base + C::kBarOff;
+  auto bar = [&](int i) -> uint32_t { return bar0 + 8u * static_cast<uint32_t>(i); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
+
+  const DenseWork w = dense_work(p);
+  const int g = w.h / p.group;
+  const Band band = band_of(p.sparse_mode, p.pre_tokens, p.next_tokens, w.sq, w.skv);
+  const TileRange tr = tile_range(w.qt, w.sq, w.skv, band);
+  const int n = tr.kt_end - tr.kt_begin;
+  const bool general_mask = (p.atten_mask != nullptr) || (p.pse != nullptr);
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    mbar_init(bar(C::kBarQFull), 1);
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(bar(C::kBarKFull + s), 1);
+      mbar_init(bar(C::kBarKEmpty + s), 1);
+      mbar_init(bar(C::kBarVFull + s), 1);
+      mbar_init(bar(C::kBarVEmpty + s), 1);
+    }
+    for (int b2 = 0; b2 < 2; ++b2) {
+      mbar_init(bar(C::kBarSFull + b2), 1);
+      mbar_init(bar(C::kBarSFree + b2), 128);
+      mbar_init(bar(C::kBarPFull + b2), 128);
+    }
+    mbar_init(bar(C::kBarPVDone), 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&p.tm_q);
+    tma_prefetch_desc(&p.tm_k);
+    tma_prefetch_desc(&p.tm_v);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0 && n > 0) {
+      const uint64_t pol_q = l2_policy_evict_first();
+      const uint64_t pol_kv = l2_policy_evict_last();
+      const int q_row = static_cast<int>(w.q_row0 + (int64_t)w.qt * kTile);
+      mbar_arrive_expect_tx(bar(C::kBarQFull), C::kTileBytes);
+      for (int sub = 0; sub < D / 64; ++sub)
+        tma_load_4d(base + C::kQOff + sub * C::kSubBytes, &p.tm_q, bar(C::kBarQFull), sub * 64, q_row, w.h,
+                    w.coord_b, pol_q);
+      for (int it = 0; it < n; ++it) {
+        const int s = it % C::kStages;
+        const uint32_t ph = (it / C::kStages) & 1;
+        const int kv_row = static_cast<int>(w.kv_row0 + (int64_t)(tr.kt_begin + it) * kTile);
+        if (it >= C::kStages && !mbar_wait(bar(C::kBarKEmpty + s), ph ^ 1, abort_flag)) break;
+        mbar_arrive_expect_tx(bar(C::kBarKFull + s), C::kTileBytes);
+        for (int sub = 0; sub < D / 64; ++sub)
+          tma_load_4d(base + C::kKOff + s * C::kTileBytes + sub * C::kSubBytes, &p.tm_k, bar(C::kBarKFull + s),
+                      sub * 64, kv_row, g, w.coord_b, pol_kv);
+        if (it >= C::kStages && !mbar_wait(bar(C::kBarVEmpty + s), ph ^ 1, abort_flag)) break;
+        mbar_arrive_expect_tx(bar(C::kBarVFull + s), C::kTileBytes);
+        for (int sub = 0; sub < D / 64; ++sub)
+          tma_load_4d(base + C::kVOff + s * C::kTileBytes + sub * C::kSubBytes, &p.tm_v, bar(C::kBarVFull + s),
+                      sub * 64, kv_row, g, w.coord_b, pol_kv);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0 && n > 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16(128, 128, false);
+      constexpr uint32_t idesc_pv = idesc_bf16(128, D, true);
+      bool ok = mbar_wait(bar(C::kBarQFull), 0, abort_flag);
+      auto issue_pv = [&](int j) -> bool {
+        const int bj = j & 1;
+        const int s = j % C::kStages;
+        if (!mbar_wait(bar(C::kBarPFull + bj), (j >> 1) & 1, abort_flag)) return false;
+        if (!mbar_wait(bar(C::kBarVFull + s), (j / C::kStages) & 1, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t vbase = base + C::kVOff + s * C::kTileBytes;
+        const uint32_t pcol = bj ? C::kColP1 : C::kColP0;
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk) {
+          // B = V tile, MN-major: 16 key rows per step (2048 B), D-halves 16 KB apart
+          const uint64_t bdesc = sdesc_sw128(vbase + kk * 2048, C::kSubBytes, 1024);
+          mma_f16_ts(tmem + C::kColO, tmem + pcol + kk * 8, bdesc, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(bar(C::kBarPVDone));
+        mma_commit(bar(C::kBarVEmpty + s));
+        return true;
+      };
+      const uint32_t qbase = base + C::kQOff;
+      for (int it = 0; ok && it < n; ++it) {
+        const int s = it % C::kStages;
+        const int bi = it & 1;
+        if (!mbar_wait(bar(C::kBarKFull + s), (it / C::kStages) & 1, abort_flag)) { ok = false; break; }
+        if (it >= 2 && !mbar_wait(bar(C::kBarSFree + bi), ((it - 2) >> 1) & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t kbase = base + C::kKOff + s * C::kTileBytes;
+        const uint32_t scol = bi ? C::kColS1 : C::kColS0;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          // A = Q, B = K, both K-major: 16 elements (32 B) per step inside a 64-wide column
+          const uint32_t off = (kk >> 2) * C::kSubBytes + (kk & 3) * 32;
+          mma_f16_ss(tmem + scol, sdesc_sw128(qbase + off, 16, 1024), sdesc_sw128(kbase + off, 16, 1024), idesc_qk,
+                     kk > 0 ? 1u : 0u);
+        }
+        mma_commit(bar(C::kBarSFull + bi));
+        mma_commit(bar(C::kBarKEmpty + s));
+        if (it >= 1 && !issue_pv(it - 1)) { ok = false; break; }
+      }
+      if (ok) issue_pv(n - 1);
+    }
+  } else {
+    // ---------------------------------------------------------------- softmax warps
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const int64_t i_loc = (int64_t)w.qt * kTile + row;  // query index inside the sequence
+    const bool has_pse = p.pse != nullptr;
+    const float vs = has_pse ? 1.0f : p.scale;  // score = value * vs
+    const float c = vs * 1.4426950408889634f;   // value -> log2 domain
+    const float kNegInf = -__int_as_float(0x7f800000);
+    // per-row band in column indices of the sequence
+    const int64_t j_lo = i_loc - band.lo_off;
+    const int64_t j_hi = min64(w.skv - 1, i_loc + band.hi_off);
+
+    const uint8_t* mrow = nullptr;
+    const __nv_bfloat16* prow = nullptr;
+    if (p.atten_mask && i_loc < w.sq)
+      mrow = p.atten_mask + w.b * p.m_batch_stride + w.h * p.m_head_stride + i_loc * p.m_row_stride;
+    if (has_pse && i_loc < w.sq)
+      prow = p.pse + w.b * p.p_batch_stride + w.h * p.p_head_stride + i_loc * p.p_row_stride;
+
+    float m_ref = kNegInf, m_true = kNegInf, l = 0.f;
+    bool ok = true;
+    for (int it = 0; it < n; ++it) {
+      const int kt = tr.kt_begin + it;
+      const int bi = it & 1;
+      if (!mbar_wait(bar(C::kBarSFull + bi), (it >> 1) & 1, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      float sv[128];
+      {
+        uint32_t r[32];
+        const uint32_t scol = tmem + lane_off + (bi ? C::kColS1 : C::kColS0);
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          tmem_ld32_wait(scol + ch * 32, r);
+#pragma unroll
+          for (int x = 0; x < 32; ++x) sv[ch * 32 + x] = __uint_as_float(r[x]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar(C::kBarSFree + bi));
+
+      const bool full = (kt >= tr.full_begin && kt < tr.full_end);
+      if (!full || general_mask) {
+        const int64_t col0 = (int64_t)kt * kTile;
+        const int64_t clo = j_lo - col0, chi = j_hi - col0;
+#pragma unroll
+        for (int x = 0; x < 128; ++x) {
+          float v = sv[x];
+          if (has_pse) {
+            const int64_t j = col0 + x;
+            v = v * p.scale + ((prow && j < w.skv) ? __bfloat162float(prow[j * 1]) : 0.f);
+          }
+          bool keep = (x >= clo) && (x <= chi);
+          if (mrow) {
+            const int64_t j = col0 + x;
+            keep = keep && (j < w.skv) && (mrow[j] == 0);
+          }
+          sv[x] = keep ? v : kNegInf;
+        }
+      }
+      float rmax = sv[0];
+#pragma unroll
+      for (int x = 1; x < 128; ++x) rmax = fmaxf(rmax, sv[x]);
+      const float m_new = fmaxf(m_true, rmax);
+      const bool upd = (m_new > m_ref) && (m_ref == kNegInf || (m_new - m_ref) * c > 8.0f);
+      const float alpha = upd ? ex2((m_ref - m_new) * c) : 1.0f;
+      const bool need = upd && (it > 0) && (m_ref != kNegInf);
+      if (__any_sync(0xffffffffu, need)) {
+        // rescale O: PV(it-1) must be complete first
+        if (!mbar_wait(bar(C::kBarPVDone), (it - 1) & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t r[32];
+#pragma unroll
+        for (int ch = 0; ch < D / 32; ++ch) {
+          const uint32_t oc = tmem + lane_off + C::kColO + ch * 32;
+          tmem_ld32_wait(oc, r);
+#pragma unroll
+          for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(__uint_as_float(r[x]) * alpha);
+          tmem_st32(oc, r);
+        }
+        tmem_st_wait();
+      }
+      if (upd) {
+        l *= alpha;
+        m_ref = m_new;
+      }
+      m_true = m_new;
+      const float mc = (m_ref == kNegInf) ? 0.f : m_ref * c;
+      uint32_t pk[64];
+      float lsum = 0.f;
+#pragma unroll
+      for (int x = 0; x < 64; ++x) {
+        const float p0 = ex2(fmaf(sv[2 * x], c, -mc));
+        const float p1 = ex2(fmaf(sv[2 * x + 1], c, -mc));
+        lsum += p0 + p1;
+        pk[x] = pack_bf16x2(p0, p1);
+      }
+      l += lsum;
+      {
+        const uint32_t pcol = tmem + lane_off + (bi ? C::kColP1 : C::kColP0);
+        uint32_t r[32];
+#pragma unroll
+        for (int x = 0; x < 32; ++x) r[x] = pk[x];
+        tmem_st32(pcol, r);
+#pragma unroll
+        for (int x = 0; x < 32; ++x) r[x] = pk[32 + x];
+        tmem_st32(pcol + 32, r);
+        tmem_st_wait();
+      }
+      tc_fence_before();
+      mbar_arrive(bar(C::kBarPFull + bi));
+    }
+
+    // ------------------------------------------------------------ epilogue
+    const bool row_valid = i_loc < w.sq;
+    bool have_o = ok && n > 0;
+    if (have_o) {
+      have_o = mbar_wait(bar(C::kBarPVDone), (n - 1) & 1, abort_flag);
+      tc_fence_after();
+    }
+    const float inv_l = (l > 0.f) ? 1.0f / l : 0.f;
+    __nv_bfloat16* orow = nullptr;
+    if (row_valid) {
+      const int64_t orow_idx = p.tnd ? (w.tok0 + i_loc) : i_loc;
+      orow = p.out + (p.tnd ? 0 : (int64_t)w.b * p.o_batch_stride) + (int64_t)w.h * p.o_head_stride +
+             orow_idx * p.o_row_stride;
+    }
+#pragma unroll
+    for (int ch = 0; ch < D / 32; ++ch) {
+      uint32_t r[32];
+      if (have_o) {
+        tmem_ld32_wait(tmem + lane_off + C::kColO + ch * 32, r);
+      } else {
+#pragma unroll
+        for (int x = 0; x < 32; ++x) r[x] = 0u;
+      }
+      if (row_valid) {
+        uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+          uint4 v;
+          v.x = pack_bf16x2(__uint_as_float(r[8 * x + 0]) * inv_l, __uint_as_float(r[8 * x + 1]) * inv_l);
+          v.y = pack_bf16x2(__uint_as_float(r[8 * x + 2]) * inv_l, __uint_as_float(r[8 * x + 3]) * inv_l);
+          v.z = pack_bf16x2(__uint_as_float(r[8 * x + 4]) * inv_l, __uint_as_float(r[8 * x + 5]) * inv_l);
+          v.w = pack_bf16x2(__uint_as_float(r[8 * x + 6]) * inv_l, __uint_as_float(r[8 * x + 7]) * inv_l);
+          dst[x] = v;
+        }
+      }
+    }
+    if (row_valid && (p.softmax_max || p.softmax_sum)) {
+      const int64_t sidx = p.tnd ? ((int64_t)w.h * p.stat_head_stride + w.tok0 + i_loc)
+                                 : ((int64_t)w.b * p.stat_batch_stride + (int64_t)w.h * p.stat_head_stride + i_loc);
+      const bool live = (m_true != kNegInf) && (l > 0.f);
+      const float smax = live ? m_true * vs : kNegInf;
+      const float ssum = live ? l * ex2((m_ref - m_true) * c) : 0.f;
+      if (p.softmax_max) p.softmax_max[sidx] = smax;
+      if (p.softmax_sum) p.softmax_sum[sidx] = ssum;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+}  // namespace qbsa

@@ -1,0 +1,429 @@
+// C ABI of libqbsa.so: argument validation, TMA tensor maps and kernel launches.
+// The contract of every entry point is documented in include/qbsa.h.
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <numeric>
+#include <string>
+#include <vector>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/qbsa.h"
+#include "attn_dense.cuh"
+#include "attn_qbsa.cuh"
+#include "quantize.cuh"
+#include "schedule.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+qbsa_status fail(qbsa_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+qbsa_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(QBSA_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr int64_t kTokenClamp = (int64_t)1 << 40;  // |pre/next| beyond this act as unbounded
+constexpr int64_t kMaxLen = ((int64_t)1 << 31) - 256;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+qbsa_status get_encoder(EncodeTiledFn* out) {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !p)
+      return fail(QBSA_ERR_CUDA, "cuTensorMapEncodeTiled is not available (%s)", cudaGetErrorString(e));
+    fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  *out = fn;
+  return QBSA_OK;
+}
+
+// 4-D tiled map over {inner, rows, heads, batch} with a {box0, 128, 1, 1} box and
+// 128-byte swizzle.  strides[] are the byte strides of dims 1..3.
+qbsa_status make_map(CUtensorMap* map, CUtensorMapDataType dt, const void* ptr, const uint64_t dims[4],
+                     const uint64_t strides[3], uint32_t box0) {
+  EncodeTiledFn enc;
+  qbsa_status st = get_encoder(&enc);
+  if (st != QBSA_OK) return st;
+  cuuint64_t gd[4] = {dims[0], dims[1], dims[2], dims[3]};
+  cuuint64_t gs[3] = {strides[0], strides[1], strides[2]};
+  cuuint32_t box[4] = {box0, 128, 1, 1};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  CUresult r = enc(map, dt, 4, const_cast<void*>(ptr), gd, gs, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(QBSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d; dims %llu %llu %llu %llu)", (int)r,
+                (unsigned long long)dims[0], (unsigned long long)dims[1], (unsigned long long)dims[2],
+                (unsigned long long)dims[3]);
+  return QBSA_OK;
+}
+
+template <typename K>
+qbsa_status set_smem(K kernel, int bytes) {
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+  return QBSA_OK;
+}
+
+qbsa_status check_launch(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, what);
+  return QBSA_OK;
+}
+
+// ------------------------------------------------------------------------------
+// attn_fwd
+// ------------------------------------------------------------------------------
+
+struct SeqInfo {
+  int q_start, q_len, kv_start, kv_len;
+};
+
+template <int D>
+qbsa_status launch_dense(qbsa::DenseParams& prm, int64_t n_work, cudaStream_t stream) {
+  using C = qbsa::DenseCfg<D>;
+  qbsa_status st = set_smem(qbsa::attn_dense_kernel<D>, C::kSmemBytes);
+  if (st != QBSA_OK) return st;
+  qbsa::attn_dense_kernel<D><<<dim3(static_cast<unsigned>(n_work)), C::kThreads, C::kSmemBytes, stream>>>(prm);
+  return check_launch("attn_dense_kernel launch");
+}
+
+}  // namespace
+
+extern "C" {
+
+int qbsa_version(void) { return 100; }
+
+const char* qbsa_last_error(void) { return g_last_error.c_str(); }
+
+qbsa_status attn_fwd(const void* q, const void* k, const void* v, int B, int Nq, int Nkv, int Sq, int Skv, int D,
+                     int head_num, qbsa_layout input_layout, const uint8_t* atten_mask, qbsa_mask_shape mask_shape,
+                     const void* pse, int pse_batch_bcast, float scale, float keep_prob, int sparse_mode,
+                     int64_t pre_tokens, int64_t next_tokens, const int64_t* actual_seq_qlen,
+                     const int64_t* actual_seq_kvlen, void* attention_out, float* softmax_max, float* softmax_sum,
+                     void* stream) {
+  // ---------------------------------------------------------------- validation
+  if (!q || !k || !v || !attention_out) return fail(QBSA_ERR_INVALID, "q, k, v and attention_out must be non-null");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(attention_out))
+    return fail(QBSA_ERR_INVALID, "q, k, v and attention_out must be 16-byte aligned");
+  if ((softmax_max && !aligned16(softmax_max)) || (softmax_sum && !aligned16(softmax_sum)))
+    return fail(QBSA_ERR_INVALID, "softmax_max / softmax_sum must be 16-byte aligned");
+  if (B < 1 || Nq < 1 || Nkv < 1 || Sq < 0 || Skv < 0) return fail(QBSA_ERR_INVALID, "B, Nq, Nkv >= 1 and Sq, Skv >= 0");
+  if (Sq > kMaxLen || Skv > kMaxLen) return fail(QBSA_ERR_UNSUPPORTED, "sequence length above %lld", (long long)kMaxLen);
+  if (head_num != Nq) return fail(QBSA_ERR_INVALID, "head_num (%d) must equal Nq (%d)", head_num, Nq);
+  if (Nq % Nkv != 0) return fail(QBSA_ERR_INVALID, "Nq (%d) must be a multiple of Nkv (%d)", Nq, Nkv);
+  if (D < 1 || D > 768) return fail(QBSA_ERR_INVALID, "D must be in [1, 768]");
+  if (D != 64 && D != 128) return fail(QBSA_ERR_UNSUPPORTED, "this build supports D = 64 or 128 (got %d)", D);
+  if (input_layout != QBSA_LAYOUT_BNSD && input_layout != QBSA_LAYOUT_BSND && input_layout != QBSA_LAYOUT_TND)
+    return fail(QBSA_ERR_INVALID, "unknown input_layout %d", (int)input_layout);
+  if (!std::isfinite(scale)) return fail(QBSA_ERR_INVALID, "scale must be finite");
+  if (!(keep_prob > 0.f && keep_prob <= 1.f)) return fail(QBSA_ERR_INVALID, "keep_prob must be in (0, 1]");
+  if (keep_prob != 1.f) return fail(QBSA_ERR_UNSUPPORTED, "dropout (keep_prob < 1) is not implemented");
+  if (sparse_mode != 0 && sparse_mode != 2 && sparse_mode != 3)
+    return fail(QBSA_ERR_UNSUPPORTED, "sparse_mode %d is not implemented (0, 2, 3 are)", sparse_mode);
+  if (mask_shape < QBSA_MASK_NONE || mask_shape > QBSA_MASK_BNSS)
+    return fail(QBSA_ERR_INVALID, "unknown mask_shape %d", (int)mask_shape);
+  if ((atten_mask == nullptr) != (mask_shape == QBSA_MASK_NONE))
+    return fail(QBSA_ERR_INVALID, "atten_mask must be given exactly when mask_shape != QBSA_MASK_NONE");
+  const bool tnd = input_layout == QBSA_LAYOUT_TND;
+  if (tnd && (atten_mask || pse)) return fail(QBSA_ERR_UNSUPPORTED, "atten_mask / pse with TND is not implemented");
+  if (tnd && (!actual_seq_qlen || !actual_seq_kvlen))
+    return fail(QBSA_ERR_INVALID, "TND needs actual_seq_qlen and actual_seq_kvlen");
+  if (!tnd && (actual_seq_qlen || actual_seq_kvlen))
+    return fail(QBSA_ERR_INVALID, "actual_seq_qlen / actual_seq_kvlen are for TND only");
+  if (tnd && B > qbsa::kMaxSeqs) return fail(QBSA_ERR_UNSUPPORTED, "TND supports at most %d sequences", qbsa::kMaxSeqs);
+  if (pse && !aligned16(pse)) return fail(QBSA_ERR_INVALID, "pse must be 16-byte aligned");
+
+  std::vector<SeqInfo> seqs;
+  if (tnd) {
+    int64_t pq = 0, pk = 0;
+    for (int b = 0; b < B; ++b) {
+      const int64_t cq = actual_seq_qlen[b], ck = actual_seq_kvlen[b];
+      if (cq < pq || ck < pk) return fail(QBSA_ERR_INVALID, "actual_seq_*len must be non-decreasing cumulative sums");
+      seqs.push_back({(int)pq, (int)(cq - pq), (int)pk, (int)(ck - pk)});
+      pq = cq;
+      pk = ck;
+    }
+    if (pq != Sq || pk != Skv)
+      return fail(QBSA_ERR_INVALID, "last actual_seq_qlen/kvlen (%lld, %lld) must equal Sq/Skv (%d, %d)",
+                  (long long)pq, (long long)pk, Sq, Skv);
+  }
+  if (Sq == 0) return QBSA_OK;  // nothing to compute
+
+  const int64_t pre = std::max(-kTokenClamp, std::min(kTokenClamp, pre_tokens));
+  const int64_t nxt = std::max(-kTokenClamp, std::min(kTokenClamp, next_tokens));
+
+  // ---------------------------------------------------------------- parameters
+  qbsa::DenseParams prm;
+  memset(&prm, 0, sizeof(prm));
+  prm.out = static_cast<__nv_bfloat16*>(attention_out);
+  prm.softmax_max = softmax_max;
+  prm.softmax_sum = softmax_sum;
+  prm.B = B;
+  prm.Nq = Nq;
+  prm.Nkv = Nkv;
+  prm.Sq = Sq;
+  prm.Skv = Skv;
+  prm.group = Nq / Nkv;
+  prm.sparse_mode = sparse_mode;
+  prm.pre_tokens = pre;
+  prm.next_tokens = nxt;
+  prm.scale = scale;
+  prm.tnd = tnd ? 1 : 0;
+  const int64_t eD = D;
+  uint64_t qd[4], kd[4], qs[3], ks[3];
+  if (input_layout == QBSA_LAYOUT_BNSD) {
+    prm.o_row_stride = eD;
+    prm.o_head_stride = (int64_t)Sq * eD;
+    prm.o_batch_stride = (int64_t)Nq * Sq * eD;
+    qd[0] = D; qd[1] = Sq; qd[2] = Nq; qd[3] = B;
+    kd[0] = D; kd[1] = Skv; kd[2] = Nkv; kd[3] = B;
+    qs[0] = eD * 2; qs[1] = (uint64_t)Sq * eD * 2; qs[2] = (uint64_t)Nq * Sq * eD * 2;
+    ks[0] = eD * 2; ks[1] = (uint64_t)Skv * eD * 2; ks[2] = (uint64_t)Nkv * Skv * eD * 2;
+  } else if (input_layout == QBSA_LAYOUT_BSND) {
+    prm.o_row_stride = (int64_t)Nq * eD;
+    prm.o_head_stride = eD;
+    prm.o_batch_stride = (int64_t)Sq * Nq * eD;
+    qd[0] = D; qd[1] = Sq; qd[2] = Nq; qd[3] = B;
+    kd[0] = D; kd[1] = Skv; kd[2] = Nkv; kd[3] = B;
+    qs[0] = (uint64_t)Nq * eD * 2; qs[1] = eD * 2; qs[2] = (uint64_t)Sq * Nq * eD * 2;
+    ks[0] = (uint64_t)Nkv * eD * 2; ks[1] = eD * 2; ks[2] = (uint64_t)Skv * Nkv * eD * 2;
+  } else {
+    prm.o_row_stride = (int64_t)Nq * eD;
+    prm.o_head_stride = eD;
+    prm.o_batch_stride = 0;
+    qd[0] = D; qd[1] = Sq; qd[2] = Nq; qd[3] = 1;
+    kd[0] = D; kd[1] = std::max(Skv, 1); kd[2] = Nkv; kd[3] = 1;
+    qs[0] = (uint64_t)Nq * eD * 2; qs[1] = eD * 2; qs[2] = (uint64_t)Sq * Nq * eD * 2;
+    ks[0] = (uint64_t)Nkv * eD * 2; ks[1] = eD * 2; ks[2] = (uint64_t)std::max(Skv, 1) * Nkv * eD * 2;
+  }
+  if (!tnd && Skv == 0) kd[1] = 1;  // map needs a non-zero extent; no tile is visited
+  if (tnd) {
+    prm.stat_head_stride = Sq;
+    prm.stat_batch_stride = 0;
+  } else {
+    prm.stat_head_stride = Sq;
+    prm.stat_batch_stride = (int64_t)Nq * Sq;
+  }
+  if (atten_mask) {
+    prm.atten_mask = atten_mask;
+    prm.m_row_stride = Skv;
+    prm.m_head_stride = (mask_shape == QBSA_MASK_BNSS) ? (int64_t)Sq * Skv : 0;
+    prm.m_batch_stride = (mask_shape == QBSA_MASK_SS) ? 0
+                         : (mask_shape == QBSA_MASK_B1SS) ? (int64_t)Sq * Skv
+                                                          : (int64_t)Nq * Sq * Skv;
+  }
+  if (pse) {
+    prm.pse = static_cast<const __nv_bfloat16*>(pse);
+    prm.p_row_stride = Skv;
+    prm.p_head_stride = (int64_t)Sq * Skv;
+    prm.p_batch_stride = pse_batch_bcast ? 0 : (int64_t)Nq * Sq * Skv;
+  }
+
+  int64_t n_rank = 0;
+  if (tnd) {
+    std::vector<int> order(B);
+    std::iota(order.begin(), order.end(), 0);
+    std::stable_sort(order.begin(), order.end(), [&](int a, int b2) { return seqs[a].q_len > seqs[b2].q_len; });
+    prm.n_seq = B;
+    int acc = 0;
+    for (int i = 0; i < B; ++i) {
+      const SeqInfo& s = seqs[order[i]];
+      prm.seq_q_start[i] = s.q_start;
+      prm.seq_q_len[i] = s.q_len;
+      prm.seq_kv_start[i] = s.kv_start;
+      prm.seq_kv_len[i] = s.kv_len;
+      prm.seq_tile_start[i] = acc;
+      acc += (s.q_len + qbsa::kTile - 1) / qbsa::kTile;
+    }
+    prm.seq_tile_start[B] = acc;
+    n_rank = acc;
+  } else {
+    prm.n_qtiles = (Sq + qbsa::kTile - 1) / qbsa::kTile;
+    n_rank = (int64_t)prm.n_qtiles * B;
+  }
+  const int64_t n_work = n_rank * Nq;
+  if (n_work == 0) return QBSA_OK;
+  if (n_work > 0x7fffffffLL) return fail(QBSA_ERR_UNSUPPORTED, "too many query tiles (%lld)", (long long)n_work);
+
+  qbsa_status st;
+  if ((st = make_map(&prm.tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, qd, qs, 64)) != QBSA_OK) return st;
+  if ((st = make_map(&prm.tm_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, k, kd, ks, 64)) != QBSA_OK) return st;
+  if ((st = make_map(&prm.tm_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, v, kd, ks, 64)) != QBSA_OK) return st;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return D == 128 ? launch_dense<128>(prm, n_work, s) : launch_dense<64>(prm, n_work, s);
+}
+
+// ------------------------------------------------------------------------------
+// qbsa_fwd
+// ------------------------------------------------------------------------------
+
+qbsa_status qbsa_fwd(const int8_t* q_i8, const int8_t* k_i8, const float* q_block_scale, const float* k_block_scale,
+                     const uint8_t* v_fp8, const float* v_channel_scale, const uint8_t* block_mask, int B, int Nq,
+                     int Nkv, int Sq, int Skv, int D, float scale, void* attention_out, float* softmax_max,
+                     float* softmax_sum, void* stream) {
+  if (!q_i8 || !k_i8 || !q_block_scale || !k_block_scale || !v_fp8 || !v_channel_scale || !block_mask ||
+      !attention_out)
+    return fail(QBSA_ERR_INVALID, "all tensor arguments except the softmax statistics must be non-null");
+  if (!aligned16(q_i8) || !aligned16(k_i8) || !aligned16(v_fp8) || !aligned16(attention_out))
+    return fail(QBSA_ERR_INVALID, "q_i8, k_i8, v_fp8 and attention_out must be 16-byte aligned");
+  if (B < 1 || Nq < 1 || Nkv < 1 || Sq < 0 || Skv < 0) return fail(QBSA_ERR_INVALID, "B, Nq, Nkv >= 1 and Sq, Skv >= 0");
+  if (Nq % Nkv != 0) return fail(QBSA_ERR_INVALID, "Nq (%d) must be a multiple of Nkv (%d)", Nq, Nkv);
+  if (D != 128) return fail(QBSA_ERR_UNSUPPORTED, "qbsa_fwd supports D = 128 (got %d)", D);
+  if (!std::isfinite(scale)) return fail(QBSA_ERR_INVALID, "scale must be finite");
+  if (Sq > kMaxLen || Skv > kMaxLen) return fail(QBSA_ERR_UNSUPPORTED, "sequence length above %lld", (long long)kMaxLen);
+  const int nqb = (Sq + 127) / 128, nkb = (Skv + 127) / 128;
+  if (nkb > qbsa::kQbsaMaxKBlocks)
+    return fail(QBSA_ERR_UNSUPPORTED, "ceil(Skv/128) = %d exceeds %d", nkb, qbsa::kQbsaMaxKBlocks);
+  if (Sq == 0) return QBSA_OK;
+
+  qbsa::QbsaParams prm;
+  memset(&prm, 0, sizeof(prm));
+  prm.q_scale = q_block_scale;
+  prm.k_scale = k_block_scale;
+  prm.v_scale = v_channel_scale;
+  prm.block_mask = block_mask;
+  prm.out = static_cast<__nv_bfloat16*>(attention_out);
+  prm.softmax_max = softmax_max;
+  prm.softmax_sum = softmax_sum;
+  prm.B = B;
+  prm.Nq = Nq;
+  prm.Nkv = Nkv;
+  prm.Sq = Sq;
+  prm.Skv = Skv;
+  prm.group = Nq / Nkv;
+  prm.nqb = nqb;
+  prm.nkb = nkb;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  const int64_t n_work = (int64_t)B * nqb * Nq;
+  if (n_work > 0x7fffffffLL) return fail(QBSA_ERR_UNSUPPORTED, "too many query blocks");
+  if (Skv == 0) {
+    // no key: every row is fully masked; keep the kernel path (no block is visited)
+  }
+  const uint64_t qd[4] = {128, (uint64_t)Sq, (uint64_t)Nq, (uint64_t)B};
+  const uint64_t kd[4] = {128, (uint64_t)std::max(Skv, 1), (uint64_t)Nkv, (uint64_t)B};
+  const uint64_t qs[3] = {128, (uint64_t)Sq * 128, (uint64_t)Nq * Sq * 128};
+  const uint64_t ks[3] = {128, (uint64_t)std::max(Skv, 1) * 128, (uint64_t)Nkv * std::max(Skv, 1) * 128};
+  qbsa_status st;
+  if ((st = make_map(&prm.tm_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, q_i8, qd, qs, 128)) != QBSA_OK) return st;
+  if ((st = make_map(&prm.tm_k, CU_TENSOR_MAP_DATA_TYPE_UINT8, k_i8, kd, ks, 128)) != QBSA_OK) return st;
+  if ((st = make_map(&prm.tm_v, CU_TENSOR_MAP_DATA_TYPE_UINT8, v_fp8, kd, ks, 128)) != QBSA_OK) return st;
+  if ((st = set_smem(qbsa::attn_qbsa_kernel, qbsa::QbsaCfg::kSmemBytes)) != QBSA_OK) return st;
+  qbsa::attn_qbsa_kernel<<<dim3(static_cast<unsigned>(n_work)), qbsa::QbsaCfg::kThreads, qbsa::QbsaCfg::kSmemBytes,
+                           static_cast<cudaStream_t>(stream)>>>(prm);
+  return check_launch("attn_qbsa_kernel launch");
+}
+
+// ------------------------------------------------------------------------------
+// quantisers
+// ------------------------------------------------------------------------------
+
+qbsa_status qbsa_quantize_qk(const void* x_bf16, int B, int N, int S, int D, int8_t* codes, float* scales,
+                             void* stream) {
+  if (!x_bf16 || !codes || !scales) return fail(QBSA_ERR_INVALID, "null pointer");
+  if (B < 1 || N < 1 || S < 1 || D < 1) return fail(QBSA_ERR_INVALID, "B, N, S, D must be >= 1");
+  const int nblk = (S + 127) / 128;
+  if (nblk > 0x7fffffff || N > 65535 || B > 65535) return fail(QBSA_ERR_UNSUPPORTED, "grid too large");
+  qbsa::quantize_qk_kernel<<<dim3(nblk, N, B), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __nv_bfloat16*>(x_bf16), N, S, D, codes, scales);
+  return check_launch("quantize_qk_kernel launch");
+}
+
+qbsa_status qbsa_quantize_v(const void* v_bf16, int B, int N, int S, int D, uint8_t* codes, float* scales,
+                            void* stream) {
+  if (!v_bf16 || !codes || !scales) return fail(QBSA_ERR_INVALID, "null pointer");
+  if (B < 1 || N < 1 || S < 1 || D < 1) return fail(QBSA_ERR_INVALID, "B, N, S, D must be >= 1");
+  if (D % 2 != 0 || D > 1024) return fail(QBSA_ERR_UNSUPPORTED, "D must be even and <= 1024");
+  if (N > 65535 || B > 65535) return fail(QBSA_ERR_UNSUPPORTED, "grid too large");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t nsc = (int64_t)B * N * D;
+  cudaError_t e = cudaMemsetAsync(scales, 0, nsc * sizeof(float), s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+  const int rows_per_cta = 256;
+  qbsa::v_colmax_kernel<<<dim3((S + rows_per_cta - 1) / rows_per_cta, N, B), D, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(v_bf16), N, S, D, rows_per_cta, reinterpret_cast<unsigned int*>(scales));
+  qbsa_status st = check_launch("v_colmax_kernel launch");
+  if (st != QBSA_OK) return st;
+  qbsa::v_scale_kernel<<<(unsigned)((nsc + 255) / 256), 256, 0, s>>>(scales, (int)nsc);
+  if ((st = check_launch("v_scale_kernel launch")) != QBSA_OK) return st;
+  const int64_t total = (int64_t)B * N * S * D;
+  qbsa::v_quant_kernel<<<148 * 8, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(v_bf16), N, S, D, scales, codes,
+                                                total);
+  return check_launch("v_quant_kernel launch");
+}
+
+// ------------------------------------------------------------------------------
+// schedule export, mask compaction hook, error word
+// ------------------------------------------------------------------------------
+
+qbsa_status attn_tile_schedule(int64_t sq, int64_t skv, int sparse_mode, int64_t pre_tokens, int64_t next_tokens,
+                               int32_t* kt_begin, int32_t* kt_end, int32_t* full_begin, int32_t* full_end,
+                               int64_t n_qtiles) {
+  if (!kt_begin || !kt_end || !full_begin || !full_end) return fail(QBSA_ERR_INVALID, "null output array");
+  if (sq < 0 || skv < 0 || sq > kMaxLen || skv > kMaxLen) return fail(QBSA_ERR_INVALID, "bad sequence lengths");
+  if (sparse_mode != 0 && sparse_mode != 2 && sparse_mode != 3)
+    return fail(QBSA_ERR_UNSUPPORTED, "sparse_mode %d is not implemented", sparse_mode);
+  if (n_qtiles != (sq + qbsa::kTile - 1) / qbsa::kTile) return fail(QBSA_ERR_INVALID, "n_qtiles must be ceil(sq/128)");
+  const int64_t pre = std::max(-kTokenClamp, std::min(kTokenClamp, pre_tokens));
+  const int64_t nxt = std::max(-kTokenClamp, std::min(kTokenClamp, next_tokens));
+  const qbsa::Band band = qbsa::band_of(sparse_mode, pre, nxt, sq, skv);
+  for (int64_t t = 0; t < n_qtiles; ++t) {
+    const qbsa::TileRange r = qbsa::tile_range((int)t, sq, skv, band);
+    kt_begin[t] = r.kt_begin;
+    kt_end[t] = r.kt_end;
+    full_begin[t] = r.full_begin;
+    full_end[t] = r.full_end;
+  }
+  return QBSA_OK;
+}
+
+qbsa_status qbsa_block_lists(const uint8_t* block_mask, int64_t rows, int n_kb, int32_t* lists, int32_t* counts,
+                             void* stream) {
+  if (!block_mask || !lists || !counts) return fail(QBSA_ERR_INVALID, "null pointer");
+  if (rows < 0 || n_kb < 1 || n_kb > qbsa::kQbsaMaxKBlocks) return fail(QBSA_ERR_INVALID, "bad rows / n_kb");
+  if (rows == 0) return QBSA_OK;
+  const int64_t grid = (rows + 3) / 4;
+  if (grid > 0x7fffffffLL) return fail(QBSA_ERR_UNSUPPORTED, "too many rows");
+  qbsa::qbsa_block_lists_kernel<<<(unsigned)grid, 128, 0, static_cast<cudaStream_t>(stream)>>>(
+      block_mask, (int)rows, n_kb, lists, counts);
+  return check_launch("qbsa_block_lists_kernel launch");
+}
+
+qbsa_status qbsa_check(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  unsigned int word = 0;
+  e = cudaMemcpyFromSymbol(&word, qbsa::g_device_error, sizeof(word));
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
+  if (word != 0) {
+    const unsigned int zero = 0;
+    cudaMemcpyToSymbol(qbsa::g_device_error, &zero, sizeof(zero));
+    return fail(QBSA_ERR_TIMEOUT, "a kernel wait exceeded its time limit (device error word %u)", word);
+  }
+  return QBSA_OK;
+}
+
+}  // extern "C"

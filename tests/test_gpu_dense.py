@@ -1,0 +1,152 @@
+"""GPU parity of attn_fwd (dense bf16) against the fp64 oracle, through the C ABI."""
+
+import numpy as np
+import pytest
+import torch
+
+import quantized_block_sparse_attn_b200 as qb
+from oracle import dense
+from workloads import (CONFIGS, bf16_bits_from_f32, blocky_qk_bf16, iid_normal_bf16, random_atten_mask,
+                       random_pse_bf16, sample_rows)
+from tests.gpu_util import (DENSE_MAX_ABS, DENSE_MEAN_ABS, compare_out, compare_stats, dev, dev_bf16, host_f64)
+
+pytestmark = pytest.mark.gpu
+INF = qb.INF_TOKENS
+
+
+def _bnsd(seed, B, Nq, Nkv, Sq, Skv, D):
+    q = iid_normal_bf16(seed, 0, B, Nq, Sq, D)
+    k = iid_normal_bf16(seed, 1, B, Nkv, Skv, D)
+    v = iid_normal_bf16(seed, 2, B, Nkv, Skv, D)
+    return q, k, v
+
+
+def _run_and_compare(q, k, v, layout, Nq, scale, mode=0, pre=INF, nxt=INF, mask=None, mask_shape=None, pse=None,
+                     cq=None, ck=None, q_rows=None, heads=None):
+    tq, tk, tv = dev_bf16(q), dev_bf16(k), dev_bf16(v)
+    tm = None if mask is None else dev(mask)
+    tp = None if pse is None else dev_bf16(pse)
+    out, smax, ssum = qb.attn_fwd(tq, tk, tv, Nq, layout, atten_mask=tm, mask_shape=mask_shape, pse=tp, scale=scale,
+                                  sparse_mode=mode, pre_tokens=pre, next_tokens=nxt, actual_seq_qlen=cq,
+                                  actual_seq_kvlen=ck)
+    qb.check()
+    ref, rmax, rsum = dense.attention_forward(q, k, v, layout=layout, scale=scale, sparse_mode=mode, pre_tokens=pre,
+                                              next_tokens=nxt, atten_mask=mask, pse=pse, actual_seq_qlen=cq,
+                                              actual_seq_kvlen=ck, q_rows=q_rows, heads=heads)
+    mx, mn = compare_out(host_f64(out), ref, DENSE_MAX_ABS, DENSE_MEAN_ABS)
+    compare_stats(smax.cpu().numpy(), ssum.cpu().numpy(), rmax, rsum)
+    return mx, mn
+
+
+@pytest.mark.parametrize("B,Nq,Nkv,Sq,Skv,D,mode,pre,nxt,layout", [
+    (1, 2, 2, 256, 256, 64, 0, INF, INF, "BNSD"),      # the tiny workload
+    (2, 4, 2, 300, 333, 128, 0, INF, INF, "BNSD"),     # ragged tails, GQA
+    (1, 2, 1, 300, 333, 128, 2, INF, INF, "BNSD"),
+    (1, 2, 1, 333, 300, 128, 3, INF, INF, "BNSD"),     # rows with no key (Skv < Sq)
+    (1, 2, 2, 300, 333, 128, 3, INF, INF, "BSND"),
+    (2, 2, 1, 520, 520, 64, 0, 100, 20, "BSND"),       # band
+    (1, 1, 1, 640, 640, 128, 0, -50, 200, "BNSD"),     # band excluding the diagonal
+    (1, 1, 1, 1, 1, 128, 0, INF, INF, "BNSD"),
+    (1, 1, 1, 1, 700, 64, 3, INF, INF, "BNSD"),
+    (1, 3, 1, 1000, 1000, 128, 2, INF, INF, "BNSD"),
+])
+def test_dense_parity(B, Nq, Nkv, Sq, Skv, D, mode, pre, nxt, layout):
+    q, k, v = _bnsd(7, B, Nq, Nkv, Sq, Skv, D)
+    if layout == "BSND":
+        q, k, v = (np.ascontiguousarray(np.swapaxes(t, 1, 2)) for t in (q, k, v))
+    _run_and_compare(q, k, v, layout, Nq, D ** -0.5, mode, pre, nxt)
+
+
+@pytest.mark.parametrize("shape", ["SS", "B1SS", "BNSS"])
+def test_dense_atten_mask(shape):
+    B, Nq, S, D = 2, 2, 200, 64
+    q, k, v = _bnsd(8, B, Nq, Nq, S, S, D)
+    mshape = {"SS": (S, S), "B1SS": (B, 1, S, S), "BNSS": (B, Nq, S, S)}[shape]
+    mask = random_atten_mask(8, mshape, 0.3)
+    _run_and_compare(q, k, v, "BNSD", Nq, 0.125, 0, 150, 150, mask=mask, mask_shape=shape)
+
+
+@pytest.mark.parametrize("bcast", [False, True])
+def test_dense_pse(bcast):
+    B, Nq, S, D = 2, 2, 200, 128
+    q, k, v = _bnsd(9, B, Nq, Nq, S, S, D)
+    pse = random_pse_bf16(9, (1 if bcast else B, Nq, S, S), 2.0)
+    _run_and_compare(q, k, v, "BNSD", Nq, D ** -0.5, 3, pse=pse)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_dense_tnd_gqa_causal(D):
+    lens_q, lens_k = [100, 300, 77, 256], [130, 300, 50, 256]
+    cq, ck = np.cumsum(lens_q), np.cumsum(lens_k)
+    Nq, Nkv = 4, 2
+    q = iid_normal_bf16(10, 0, 1, 1, cq[-1], Nq * D).reshape(cq[-1], Nq, D)
+    k = iid_normal_bf16(10, 1, 1, 1, ck[-1], Nkv * D).reshape(ck[-1], Nkv, D)
+    v = iid_normal_bf16(10, 2, 1, 1, ck[-1], Nkv * D).reshape(ck[-1], Nkv, D)
+    _run_and_compare(q, k, v, "TND", Nq, D ** -0.5, 3, cq=cq, ck=ck)
+
+
+@pytest.mark.parametrize("mode,pre,nxt,layout", [(0, 300, 40, "BNSD"), (2, INF, INF, "BNSD"), (3, INF, INF, "BSND"),
+                                                 (3, INF, INF, "TND")])
+def test_mask_logic_bit_exact_via_zero_query(mode, pre, nxt, layout):
+    """Q = 0 makes every kept weight exactly 1: softmax_sum must equal the kept-key count."""
+    D, Nq, Nkv = 128, 2, 1
+    if layout == "TND":
+        lens_q, lens_k = [333, 129, 500], [400, 129, 257]
+        cq, ck = np.cumsum(lens_q), np.cumsum(lens_k)
+        q = np.zeros((cq[-1], Nq, D), dtype=np.uint16)
+        k = iid_normal_bf16(11, 1, 1, 1, ck[-1], Nkv * D).reshape(ck[-1], Nkv, D)
+        v = iid_normal_bf16(11, 2, 1, 1, ck[-1], Nkv * D).reshape(ck[-1], Nkv, D)
+    else:
+        cq = ck = None
+        Sq, Skv = 700, 531
+        q = np.zeros((1, Nq, Sq, D), dtype=np.uint16)
+        _, k, v = _bnsd(11, 1, Nq, Nkv, Sq, Skv, D)
+        if layout == "BSND":
+            q, k, v = (np.ascontiguousarray(np.swapaxes(t, 1, 2)) for t in (q, k, v))
+    out, smax, ssum = qb.attn_fwd(dev_bf16(q), dev_bf16(k), dev_bf16(v), Nq, layout, scale=0.3, sparse_mode=mode,
+                                  pre_tokens=pre, next_tokens=nxt, actual_seq_qlen=cq, actual_seq_kvlen=ck)
+    qb.check()
+    ssum = ssum.cpu().numpy()
+    if layout == "TND":
+        for b in range(len(cq)):
+            q0, q1 = (cq[b - 1] if b else 0), cq[b]
+            cnt = dense.allowed(q1 - q0, lens_k[b], mode, pre, nxt).sum(axis=1)
+            for h in range(Nq):
+                assert np.array_equal(ssum[h, q0:q1], cnt.astype(np.float32))
+    else:
+        cnt = dense.allowed(700, 531, mode, pre, nxt).sum(axis=1)
+        for h in range(Nq):
+            assert np.array_equal(ssum[0, h], cnt.astype(np.float32))
+
+
+def test_causal_workload_sampled():
+    c = CONFIGS["causal"]
+    B, N, S, D = c["B"], c["Nq"], c["S"], c["D"]
+    q, k, v = _bnsd(c["seed"], B, N, N, S, S, D)
+    rows = np.concatenate([np.arange(qb_ * 128, qb_ * 128 + 128) for qb_ in sample_rows(c["seed"], S, 4)])
+    _run_and_compare(q, k, v, "BNSD", N, c["scale"], 3, q_rows=rows)
+
+
+def test_gqa_varlen_workload_sampled():
+    c = CONFIGS["gqa_varlen"]
+    lens = list(c["seqlens"])
+    cq = np.cumsum(lens)
+    T, Nq, Nkv, D = cq[-1], c["Nq"], c["Nkv"], c["D"]
+    q = iid_normal_bf16(c["seed"], 0, 1, 1, T, Nq * D).reshape(T, Nq, D)
+    k = iid_normal_bf16(c["seed"], 1, 1, 1, T, Nkv * D).reshape(T, Nkv, D)
+    v = iid_normal_bf16(c["seed"], 2, 1, 1, T, Nkv * D).reshape(T, Nkv, D)
+    rows = np.array(sorted(set(range(0, 128)) | set(range(1000, 1024)) | set(range(4000, 4100)) |
+                           set(range(10232, 10360))))
+    _run_and_compare(q, k, v, "TND", Nq, c["scale"], 3, cq=cq, ck=cq, q_rows=rows, heads=None)
+
+
+@pytest.mark.slow
+def test_video_workload_sampled():
+    c = CONFIGS["video"]
+    N, S, D = c["Nq"], c["S"], c["D"]
+    heads = [0, 17, 39]
+    q = blocky_qk_bf16(c["seed"], "q", 1, N, S, D)
+    k = blocky_qk_bf16(c["seed"], "k", 1, N, S, D)
+    v = iid_normal_bf16(c["seed"], 2, 1, N, S, D)
+    rows = np.concatenate([np.arange(b * 128, b * 128 + 128) for b in sample_rows(c["seed"], S, 4)])
+    _run_and_compare(q, k, v, "BNSD", N, c["scale"], 0, q_rows=rows, heads=[(0, h) for h in heads])

@@ -1,0 +1,145 @@
+"""GPU parity of qbsa_fwd and the on-GPU quantisers against the oracle, through the C ABI."""
+
+import numpy as np
+import pytest
+import torch
+
+import quantized_block_sparse_attn_b200 as qb
+from oracle import dense, quant
+from workloads import CONFIGS, block_keep_mask, blocky_qk_bf16, iid_normal_bf16, sample_rows
+from tests.gpu_util import QUANT_MAX_ABS, compare_out, compare_stats, dev, dev_bf16, host_f64
+
+pytestmark = pytest.mark.gpu
+
+
+def _quantized(q, k, v):
+    q8, qs = quant.quantize_qk_per_block(q)
+    k8, ks = quant.quantize_qk_per_block(k)
+    v8, vs = quant.quantize_v_per_channel(v)
+    return q8, qs, k8, ks, v8, vs
+
+
+def _run(q8, qs, k8, ks, v8, vs, bm, scale):
+    out, smax, ssum = qb.qbsa_fwd(dev(q8), dev(k8), dev(qs), dev(ks), dev(v8), dev(vs), dev(bm), scale)
+    qb.check()
+    return host_f64(out), smax.cpu().numpy(), ssum.cpu().numpy()
+
+
+@pytest.mark.parametrize("B,Nq,Nkv,Sq,Skv,keep", [
+    (1, 2, 1, 300, 400, 0.5),     # ragged tails on both axes, GQA
+    (1, 2, 2, 1024, 1024, 0.25),
+    (2, 2, 1, 128, 640, 1.0),
+    (1, 1, 1, 1, 129, 1.0),
+])
+def test_qbsa_parity_small(B, Nq, Nkv, Sq, Skv, keep):
+    D = 128
+    q = iid_normal_bf16(20, 0, B, Nq, Sq, D)
+    k = iid_normal_bf16(20, 1, B, Nkv, Skv, D)
+    v = iid_normal_bf16(20, 2, B, Nkv, Skv, D)
+    q8, qs, k8, ks, v8, vs = _quantized(q, k, v)
+    bm = block_keep_mask(20, B, Nq, -(-Sq // 128), -(-Skv // 128), keep)
+    scale = D ** -0.5
+    got, gmax, gsum = _run(q8, qs, k8, ks, v8, vs, bm, scale)
+    ref, rmax, rsum = quant.qbsa_forward(q8, k8, qs, ks, v8, vs, bm, scale)
+    compare_out(got, ref, QUANT_MAX_ABS)
+    compare_stats(gmax, gsum, rmax, rsum)
+
+
+def test_qbsa_empty_rows_and_zero_query_counts():
+    """q = 0 gives p8 = 1 for every kept key: softmax_sum must be the exact kept-column count."""
+    B, Nq, Nkv, Sq, Skv, D = 1, 2, 1, 384, 333, 128
+    k = iid_normal_bf16(21, 1, B, Nkv, Skv, D)
+    v = iid_normal_bf16(21, 2, B, Nkv, Skv, D)
+    k8, ks = quant.quantize_qk_per_block(k)
+    v8, vs = quant.quantize_v_per_channel(v)
+    q8 = np.zeros((B, Nq, Sq, D), dtype=np.int8)
+    qs = np.ones((B, Nq, 3), dtype=np.float32)
+    bm = block_keep_mask(21, B, Nq, 3, 3, 0.67)
+    bm[0, 1, 2, :] = 0  # a query block with no kept key block
+    got, gmax, gsum = _run(q8, qs, k8, ks, v8, vs, bm, 0.1)
+    for h in range(Nq):
+        for qb_ in range(3):
+            cols = sum(min(Skv, kb * 128 + 128) - kb * 128 for kb in np.nonzero(bm[0, h, qb_])[0])
+            assert np.all(gsum[0, h, qb_ * 128:(qb_ + 1) * 128] == np.float32(cols))
+            if cols == 0:
+                assert np.all(got[0, h, qb_ * 128:(qb_ + 1) * 128] == 0)
+                assert np.all(np.isneginf(gmax[0, h, qb_ * 128:(qb_ + 1) * 128]))
+            else:
+                assert np.all(gmax[0, h, qb_ * 128:(qb_ + 1) * 128] == 0)
+
+
+def test_block_lists_hook_bit_exact():
+    rng = np.random.default_rng(22)
+    for n_kb in (1, 31, 32, 33, 512, 2048):
+        rows = (rng.random((9, n_kb)) < 0.3).astype(np.uint8)
+        rows[0] = 0
+        rows[1] = 1
+        lists, counts = qb.block_lists(dev(rows))
+        lists, counts = lists.cpu().numpy(), counts.cpu().numpy()
+        for r in range(9):
+            idx = np.nonzero(rows[r])[0]
+            assert counts[r] == len(idx)
+            assert np.array_equal(lists[r, :len(idx)], idx)
+            assert np.all(lists[r, len(idx):] == -1)
+
+
+@pytest.mark.parametrize("S", [300, 4096])
+def test_quantisers_bit_exact(S):
+    B, N, D = 2, 3, 128
+    x = blocky_qk_bf16(23, "q", B, N, S, D)
+    v = iid_normal_bf16(23, 2, B, N, S, D)
+    v[0, 1, :, 5] = 0  # an all-zero channel takes scale 1
+    c8, cs = qb.quantize_qk(dev_bf16(x))
+    v8, vs = qb.quantize_v(dev_bf16(v))
+    torch.cuda.synchronize()
+    r8, rs = quant.quantize_qk_per_block(x)
+    rv8, rvs = quant.quantize_v_per_channel(v)
+    assert np.array_equal(c8.cpu().numpy(), r8)
+    assert np.array_equal(cs.cpu().numpy().view(np.uint32), rs.view(np.uint32))
+    assert np.array_equal(vs.cpu().numpy().view(np.uint32), rvs.view(np.uint32))
+    assert np.array_equal(v8.cpu().numpy(), rv8)
+
+
+def _qbsa_workload(S, keep, heads_for_oracle, n_qblocks):
+    c = CONFIGS["qbsa"]
+    N, D, seed = c["Nq"], c["D"], c["seed"]
+    q = blocky_qk_bf16(seed, "q", 1, N, S, D)
+    k = blocky_qk_bf16(seed, "k", 1, N, S, D)
+    v = iid_normal_bf16(seed, 2, 1, N, S, D)
+    nb = S // 128
+    bm = block_keep_mask(seed, 1, N, nb, nb, keep)
+    # GPU path: quantise on the GPU (checked bit-exact against the oracle on the sampled heads)
+    tq8, tqs = qb.quantize_qk(dev_bf16(q))
+    tk8, tks = qb.quantize_qk(dev_bf16(k))
+    tv8, tvs = qb.quantize_v(dev_bf16(v))
+    out, smax, ssum = qb.qbsa_fwd(tq8, tk8, tqs, tks, tv8, tvs, dev(bm), c["scale"])
+    qb.check()
+    got, gmax, gsum = host_f64(out), smax.cpu().numpy(), ssum.cpu().numpy()
+    qbs = sample_rows(seed, S, n_qblocks)
+    for h in heads_for_oracle:
+        sl = (slice(0, 1), slice(h, h + 1))
+        q8, qs, k8, ks, v8, vs = _quantized(q[sl], k[sl], v[sl])
+        assert np.array_equal(tq8[0, h].cpu().numpy(), q8[0, 0])
+        assert np.array_equal(tk8[0, h].cpu().numpy(), k8[0, 0])
+        assert np.array_equal(tv8[0, h].cpu().numpy(), v8[0, 0])
+        assert np.array_equal(tvs[0, h].cpu().numpy().view(np.uint32), vs[0, 0].view(np.uint32))
+        ref, rmax, rsum = quant.qbsa_forward(q8, k8, qs, ks, v8, vs, bm[:, h:h + 1], c["scale"], q_blocks=qbs)
+        compare_out(got[:, h:h + 1], ref, QUANT_MAX_ABS)
+        compare_stats(gmax[:, h:h + 1], gsum[:, h:h + 1], rmax, rsum)
+        # reported, not gated: error against the unquantised attention over the same kept blocks
+        rows = np.concatenate([np.arange(b_ * 128, b_ * 128 + 128) for b_ in qbs])
+        keep_el = np.repeat(np.repeat(bm[0, h], 128, axis=0), 128, axis=1)
+        dref, _, _ = dense.attention_forward(q[sl], k[sl], v[sl], layout="BNSD", scale=c["scale"],
+                                             atten_mask=(keep_el == 0).astype(np.uint8), q_rows=rows)
+        e = np.abs(got[0, h, rows] - dref[0, 0, rows])
+        print(f"S={S} keep={keep} head {h}: error vs unquantised attention max {e.max():.3e} mean {e.mean():.3e}")
+
+
+@pytest.mark.parametrize("keep", [0.1, 0.5])
+def test_qbsa_workload_8k_sampled(keep):
+    _qbsa_workload(8192, keep, heads_for_oracle=[0, 39], n_qblocks=6)
+
+
+@pytest.mark.slow
+def test_qbsa_workload_64k_sampled():
+    _qbsa_workload(65536, 0.1, heads_for_oracle=[0, 21], n_qblocks=4)

@@ -17,4 +17,6 @@ from .gen import (  # noqa: F401
     sample_rows,
     random_atten_mask,
     random_pse_bf16,
+    device_iid_normal_bf16,
+    device_blocky_qk_bf16,
 )

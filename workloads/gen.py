@@ -133,3 +133,33 @@ def sample_rows(seed: int, n_rows: int, n_q_blocks_per_head: int = 8):
             break
         pick.add(int(e))
     return sorted(pick)
+
+
+# --------------------------------------------------------------------------------------
+# device-side generation (bench sizes): same recipes, torch's seeded CUDA generator
+# --------------------------------------------------------------------------------------
+
+def _torch_gen(seed: int, tensor_id: int, device):
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(int(np.random.SeedSequence((seed, tensor_id)).generate_state(1, dtype=np.uint64)[0] >> 1))
+    return g
+
+
+def device_iid_normal_bf16(seed: int, tensor_id: int, shape, device):
+    """bf16 tensor of iid N(0,1) draws made on the device (torch Philox generator)."""
+    import torch
+    g = _torch_gen(seed, tensor_id, device)
+    return torch.randn(shape, generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
+
+
+def device_blocky_qk_bf16(seed: int, which: str, n_batch: int, n_head: int, rows: int, d: int, device,
+                          noise_std: float = 0.3):
+    """Device-made version of ``blocky_qk_bf16`` (same recipe, different random stream)."""
+    import torch
+    tid, mid = (_Q, _MU_Q) if which == "q" else (_K, _MU_K)
+    nblk = -(-rows // BLK)
+    mu = torch.randn((n_batch, n_head, nblk, 1, d), generator=_torch_gen(seed, mid, device), device=device)
+    x = torch.randn((n_batch, n_head, nblk, BLK, d), generator=_torch_gen(seed, tid, device), device=device)
+    x.mul_(noise_std).add_(mu)
+    return x.reshape(n_batch, n_head, nblk * BLK, d)[:, :, :rows].to(torch.bfloat16).contiguous()
