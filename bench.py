@@ -42,6 +42,7 @@ def parse():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--seq", type=int, default=65536)
     p.add_argument("--keep", type=float, default=0.1)
+    p.add_argument("--dense-seq", type=int, default=61440)
     p.add_argument("--sweep", action="store_true")
     p.add_argument("--no-dense", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
@@ -360,7 +361,7 @@ def run_ours(args):
     torch.cuda.empty_cache()
     # ---------------------------------------------------------------- dense bf16 video workload
     if not args.no_dense:
-        extra["dense_video"] = dense_line(device, stream, 61440, max(2, args.warmup), 3, bf16_peak, dist)
+        extra["dense_video"] = dense_line(device, stream, args.dense_seq, max(2, args.warmup), 3, bf16_peak, dist)
     if args.sweep:
         for S in (8192, 16384, 32768, 65536, 131072):
             for keep in (0.1, 0.5):

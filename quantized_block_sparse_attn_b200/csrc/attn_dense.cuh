@@ -78,7 +78,8 @@ struct DenseCfg {
   static constexpr int kBarSFree = kBarSFull + 2;         // 2
   static constexpr int kBarPFull = kBarSFree + 2;         // 2
   static constexpr int kBarPVDone = kBarPFull + 2;        // 1
-  static constexpr int kNumBars = kBarPVDone + 1;
+  static constexpr int kBarOFinal = kBarPVDone + 1;       // 1: last P·V done (single use)
+  static constexpr int kNumBars = kBarOFinal + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   // + alignment slack; at least 120 KB so that one CTA holds an SM (and its 512 TMEM columns)
   static constexpr int kSmemUsed = kMiscOff + 16 + 1024;
@@ -169,6 +170,7 @@ __global__ void __launch_bounds__(192, 1) attn_dense_kernel(const __grid_constan
       mbar_init(bar(C::kBarPFull + b2), 128);
     }
     mbar_init(bar(C::kBarPVDone), 1);
+    mbar_init(bar(C::kBarOFinal), 1);
     fence_mbar_init();
     tma_prefetch_desc(&p.tm_q);
     tma_prefetch_desc(&p.tm_k);
@@ -253,7 +255,7 @@ __global__ void __launch_bounds__(192, 1) attn_dense_kernel(const __grid_constan
         mma_commit(bar(C::kBarKEmpty + s));
         if (it >= 1 && !issue_pv(it - 1)) { ok = false; break; }
       }
-      if (ok) issue_pv(n - 1);
+      if (ok && issue_pv(n - 1)) mma_commit(bar(C::kBarOFinal));
     }
   } else {
     // ---------------------------------------------------------------- softmax warps
@@ -373,7 +375,8 @@ __global__ void __launch_bounds__(192, 1) attn_dense_kernel(const __grid_constan
     const bool row_valid = i_loc < w.sq;
     bool have_o = ok && n > 0;
     if (have_o) {
-      have_o = mbar_wait(bar(C::kBarPVDone), (n - 1) & 1, abort_flag);
+      // a dedicated single-use barrier: pv_done's parity cannot tell PV(n-1) from PV(n-3)
+      have_o = mbar_wait(bar(C::kBarOFinal), 0, abort_flag);
       tc_fence_after();
     }
     const float inv_l = (l > 0.f) ? 1.0f / l : 0.f;

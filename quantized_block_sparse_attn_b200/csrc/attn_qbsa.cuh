@@ -64,7 +64,8 @@ struct QbsaCfg {
   static constexpr int kBarSFree = kBarSFull + 2;
   static constexpr int kBarPFull = kBarSFree + 2;
   static constexpr int kBarPVDone = kBarPFull + 2;
-  static constexpr int kNumBars = kBarPVDone + 1;
+  static constexpr int kBarOFinal = kBarPVDone + 1;  // last P·V done (single use)
+  static constexpr int kNumBars = kBarOFinal + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // tmem addr, abort flag, list count
   static constexpr int kSmemBytes = kMiscOff + 16 + 1024;
   static constexpr uint32_t kTmemCols = 512;
@@ -126,6 +127,7 @@ __global__ void __launch_bounds__(192, 1) attn_qbsa_kernel(const __grid_constant
         mbar_init(bar(C::kBarPFull + b2), 128);
       }
       mbar_init(bar(C::kBarPVDone), 1);
+      mbar_init(bar(C::kBarOFinal), 1);
       fence_mbar_init();
       tma_prefetch_desc(&p.tm_q);
       tma_prefetch_desc(&p.tm_k);
@@ -211,7 +213,7 @@ __global__ void __launch_bounds__(192, 1) attn_qbsa_kernel(const __grid_constant
         mma_commit(bar(C::kBarKEmpty + s));
         if (it >= 1 && !issue_pv(it - 1)) { ok = false; break; }
       }
-      if (ok) issue_pv(n - 1);
+      if (ok && issue_pv(n - 1)) mma_commit(bar(C::kBarOFinal));
     }
   } else {
     // ---------------------------------------------------------------- softmax warps
@@ -298,7 +300,8 @@ __global__ void __launch_bounds__(192, 1) attn_qbsa_kernel(const __grid_constant
     const bool row_valid = i_glob < p.Sq;
     bool have_o = ok && n > 0;
     if (have_o) {
-      have_o = mbar_wait(bar(C::kBarPVDone), (n - 1) & 1, abort_flag);
+      // a dedicated single-use barrier: pv_done's parity cannot tell PV(n-1) from PV(n-3)
+      have_o = mbar_wait(bar(C::kBarOFinal), 0, abort_flag);
       tc_fence_after();
     }
     float l = 0.f;

@@ -57,6 +57,14 @@ def test_dense_parity(B, Nq, Nkv, Sq, Skv, D, mode, pre, nxt, layout):
     _run_and_compare(q, k, v, layout, Nq, D ** -0.5, mode, pre, nxt)
 
 
+def test_dense_short_k_loops_repeated():
+    """Two to three K tiles per CTA, repeated: the last-P·V wait must not pass early."""
+    for rep in range(8):
+        for S, D in ((256, 64), (256, 128), (384, 64), (384, 128)):
+            q, k, v = _bnsd(30 + rep, 1, 1, 1, S, S, D)
+            _run_and_compare(q, k, v, "BNSD", 1, D ** -0.5)
+
+
 @pytest.mark.parametrize("shape", ["SS", "B1SS", "BNSS"])
 def test_dense_atten_mask(shape):
     B, Nq, S, D = 2, 2, 200, 64

@@ -45,6 +45,21 @@ def test_qbsa_parity_small(B, Nq, Nkv, Sq, Skv, keep):
     compare_stats(gmax, gsum, rmax, rsum)
 
 
+def test_qbsa_short_loops_repeated():
+    """Two or three kept blocks per query block, repeated: the last-P·V wait must not pass early."""
+    D = 128
+    for rep in range(6):
+        for S in (256, 384):
+            q = iid_normal_bf16(40 + rep, 0, 1, 1, S, D)
+            k = iid_normal_bf16(40 + rep, 1, 1, 1, S, D)
+            v = iid_normal_bf16(40 + rep, 2, 1, 1, S, D)
+            q8, qs, k8, ks, v8, vs = _quantized(q, k, v)
+            bm = np.ones((1, 1, S // 128, S // 128), dtype=np.uint8)
+            got, gmax, gsum = _run(q8, qs, k8, ks, v8, vs, bm, D ** -0.5)
+            ref, rmax, rsum = quant.qbsa_forward(q8, k8, qs, ks, v8, vs, bm, D ** -0.5)
+            compare_out(got, ref, QUANT_MAX_ABS)
+
+
 def test_qbsa_empty_rows_and_zero_query_counts():
     """q = 0 gives p8 = 1 for every kept key: softmax_sum must be the exact kept-column count."""
     B, Nq, Nkv, Sq, Skv, D = 1, 2, 1, 384, 333, 128
