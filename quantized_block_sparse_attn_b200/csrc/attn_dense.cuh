@@ -7,17 +7,22 @@
 // varlen TND follows §4.3, GQA follows §7, and the outputs are attention_out,
 // softmax_max and softmax_sum (§5).
 //
-// CTA = 6 warps:
+// CTA = 10 warps:
 //   warp 0      TMA producer: Q once, then K/V tiles into a 2-stage ring each.
 //   warp 1      TMEM owner + MMA issuer (one thread): S = Q Kᵀ (kind::f16, SS) into a
 //               double-buffered f32 TMEM tile, then O += P V (kind::f16, A = P from
 //               TMEM, B = V from shared memory, MN-major).
-//   warps 2..5  softmax: thread t owns query row 32*(warp%4)+lane (its TMEM lane),
-//               loads its S row, masks, keeps the running max, rescales O in TMEM
-//               only when the max grew by more than 2^8 (the output is unchanged
-//               by the lagging reference; the statistics are corrected at the end),
-//               writes P as bf16 into TMEM and finally normalises O and stores it.
+//   warps 2..9  softmax: query row 32*(warp%4)+lane (the warp's TMEM lane quarter);
+//               warps 2..5 own score columns [0,64), warps 6..9 columns [64,128) of
+//               the same rows, and exchange their partial row maxima through shared
+//               memory (a 64-thread named barrier per lane quarter).  O is rescaled in
+//               TMEM only when the running max grew by more than 2^8 (the lagging
+//               reference cancels in O / l; the statistics are corrected at the end).
+//               P goes to TMEM as bf16; the epilogue normalises O and stores it.
 // TMEM columns: S0 [0,128) S1 [128,256) O [256,256+D) P0 [384,448) P1 [448,512).
+//
+// CTA order: query heads are taken in groups whose K/V fit in about 48 MB of L2; in
+// a group the heaviest query tiles (causal) come first, heads fastest.
 #pragma once
 
 #include <cstdint>
@@ -47,8 +52,10 @@ struct DenseParams {
   int64_t pre_tokens, next_tokens;
   int B, Nq, Nkv, Sq, Skv, group;
   int sparse_mode;
-  int tnd;       // 1: varlen TND
-  int n_qtiles;  // BNSD/BSND: ceil(Sq/128)
+  int tnd;        // 1: varlen TND
+  int n_qtiles;   // BNSD/BSND: ceil(Sq/128)
+  int n_rank;     // query tiles per head (all batches / sequences)
+  int head_grp;   // query heads per L2 group
   float scale;
   // TND tables (sequences in processing order)
   int n_seq;
@@ -67,7 +74,8 @@ struct DenseCfg {
   static constexpr int kQOff = 0;
   static constexpr int kKOff = kQOff + kTileBytes;
   static constexpr int kVOff = kKOff + kStages * kTileBytes;
-  static constexpr int kBarOff = kVOff + kStages * kTileBytes;
+  static constexpr int kXOff = kVOff + kStages * kTileBytes;  // row-max exchange: float [2][2][128]
+  static constexpr int kBarOff = kXOff + 2 * 2 * 128 * 4;
   // barriers
   static constexpr int kBarQFull = 0;
   static constexpr int kBarKFull = 1;
@@ -87,7 +95,8 @@ struct DenseCfg {
   // TMEM columns
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256, kColP0 = 384, kColP1 = 448;
-  static constexpr int kThreads = 192;
+  static constexpr int kThreads = 320;
+  static constexpr int kSoftmaxThreads = 256;
 };
 
 struct DenseWork {
@@ -101,13 +110,18 @@ struct DenseWork {
 
 __device__ __forceinline__ DenseWork dense_work(const DenseParams& p) {
   DenseWork w;
-  // 1-D grid: heads fastest, so the first wave holds the heaviest tile of every head
-  w.h = static_cast<int>(blockIdx.x % p.Nq);
-  const int r = static_cast<int>(blockIdx.x / p.Nq);
+  // head groups (L2 reuse of K/V), heaviest query tiles first, heads fastest inside a group
+  const int64_t per_group = (int64_t)p.head_grp * p.n_rank;
+  const int grp = static_cast<int>(blockIdx.x / per_group);
+  const int h0 = grp * p.head_grp;
+  const int hcount = min(p.head_grp, p.Nq - h0);
+  const int off = static_cast<int>(blockIdx.x - grp * per_group);
+  const int r = off / hcount;
+  w.h = h0 + off % hcount;
   if (!p.tnd) {
     const int rank = r / p.B;
     w.b = r % p.B;
-    w.qt = p.n_qtiles - 1 - rank;  // heaviest (causal) tiles first
+    w.qt = p.n_qtiles - 1 - rank;
     w.q_row0 = 0;
     w.kv_row0 = 0;
     w.coord_b = w.b;
@@ -133,9 +147,14 @@ __device__ __forceinline__ DenseWork dense_work(const DenseParams& p) {
   return w;
 }
 
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 template <int D>
-__global__ void __launch_bounds__(192, 1) attn_dense_kernel(const __grid_constant__ DenseParams p) {
+__global__ void __launch_bounds__(320, 1) attn_dense_kernel(const __grid_constant__ DenseParams p) {
   using C = DenseCfg<D>;
+  constexpr int kHalfD = D / 2;  // O columns per softmax half
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
   const uint32_t base = (raw_base + 1023u) & ~1023u;
@@ -147,6 +166,7 @@ __global__ void __launch_bounds__(192, 1) attn_dense_kernel(const __grid_constan
   auto bar = [&](int i) -> uint32_t { return bar0 + 8u * static_cast<uint32_t>(i); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
+  float* xch = reinterpret_cast<float*>(smem + C::kXOff);  // [slot][half][row]
 
   const DenseWork w = dense_work(p);
   const int g = w.h / p.group;
@@ -166,8 +186,8 @@ __global__ void __launch_bounds__(192, 1) attn_dense_kernel(const __grid_constan
     }
     for (int b2 = 0; b2 < 2; ++b2) {
       mbar_init(bar(C::kBarSFull + b2), 1);
-      mbar_init(bar(C::kBarSFree + b2), 128);
-      mbar_init(bar(C::kBarPFull + b2), 128);
+      mbar_init(bar(C::kBarSFree + b2), C::kSoftmaxThreads);
+      mbar_init(bar(C::kBarPFull + b2), C::kSoftmaxThreads);
     }
     mbar_init(bar(C::kBarPVDone), 1);
     mbar_init(bar(C::kBarOFinal), 1);
@@ -260,6 +280,7 @@ __global__ void __launch_bounds__(192, 1) attn_dense_kernel(const __grid_constan
   } else {
     // ---------------------------------------------------------------- softmax warps
     const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;  // 0: score columns [0,64), 1: [64,128)
     const int row = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const int64_t i_loc = (int64_t)w.qt * kTile + row;  // query index inside the sequence
@@ -267,9 +288,9 @@ __global__ void __launch_bounds__(192, 1) attn_dense_kernel(const __grid_constan
     const float vs = has_pse ? 1.0f : p.scale;  // score = value * vs
     const float c = vs * 1.4426950408889634f;   // value -> log2 domain
     const float kNegInf = -__int_as_float(0x7f800000);
-    // per-row band in column indices of the sequence
-    const int64_t j_lo = i_loc - band.lo_off;
+    const int64_t j_lo = i_loc - band.lo_off;   // per-row band, column indices of the sequence
     const int64_t j_hi = min64(w.skv - 1, i_loc + band.hi_off);
+    const uint32_t o_col = tmem + lane_off + C::kColO + half * kHalfD;
 
     const uint8_t* mrow = nullptr;
     const __nv_bfloat16* prow = nullptr;
@@ -278,19 +299,21 @@ __global__ void __launch_bounds__(192, 1) attn_dense_kernel(const __grid_constan
     if (has_pse && i_loc < w.sq)
       prow = p.pse + w.b * p.p_batch_stride + w.h * p.p_head_stride + i_loc * p.p_row_stride;
 
-    float m_ref = kNegInf, m_true = kNegInf, l = 0.f;
+    float m_ref = kNegInf, m_true = kNegInf, l = 0.f;  // l: this half's partial sum
     bool ok = true;
     for (int it = 0; it < n; ++it) {
       const int kt = tr.kt_begin + it;
       const int bi = it & 1;
-      if (!mbar_wait(bar(C::kBarSFull + bi), (it >> 1) & 1, abort_flag)) { ok = false; break; }
+      // never leave the loop early: the paired warp waits on named barriers below, so
+      // after a failed (timed-out) wait the remaining iterations run without waiting
+      if (ok) ok = mbar_wait(bar(C::kBarSFull + bi), (it >> 1) & 1, abort_flag);
       tc_fence_after();
-      float sv[128];
+      float sv[64];
       {
         uint32_t r[32];
-        const uint32_t scol = tmem + lane_off + (bi ? C::kColS1 : C::kColS0);
+        const uint32_t scol = tmem + lane_off + (bi ? C::kColS1 : C::kColS0) + half * 64;
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
+        for (int ch = 0; ch < 2; ++ch) {
           tmem_ld32_wait(scol + ch * 32, r);
 #pragma unroll
           for (int x = 0; x < 32; ++x) sv[ch * 32 + x] = __uint_as_float(r[x]);
@@ -301,14 +324,14 @@ __global__ void __launch_bounds__(192, 1) attn_dense_kernel(const __grid_constan
 
       const bool full = (kt >= tr.full_begin && kt < tr.full_end);
       if (!full || general_mask) {
-        const int64_t col0 = (int64_t)kt * kTile;
+        const int64_t col0 = (int64_t)kt * kTile + half * 64;
         const int64_t clo = j_lo - col0, chi = j_hi - col0;
 #pragma unroll
-        for (int x = 0; x < 128; ++x) {
+        for (int x = 0; x < 64; ++x) {
           float v = sv[x];
           if (has_pse) {
             const int64_t j = col0 + x;
-            v = v * p.scale + ((prow && j < w.skv) ? __bfloat162float(prow[j * 1]) : 0.f);
+            v = v * p.scale + ((prow && j < w.skv) ? __bfloat162float(prow[j]) : 0.f);
           }
           bool keep = (x >= clo) && (x <= chi);
           if (mrow) {
@@ -318,25 +341,30 @@ __global__ void __launch_bounds__(192, 1) attn_dense_kernel(const __grid_constan
           sv[x] = keep ? v : kNegInf;
         }
       }
-      float rmax = sv[0];
+      float pmax = sv[0];
 #pragma unroll
-      for (int x = 1; x < 128; ++x) rmax = fmaxf(rmax, sv[x]);
+      for (int x = 1; x < 64; ++x) pmax = fmaxf(pmax, sv[x]);
+      // combine the two halves of the row
+      float* slot = xch + (it & 1) * 256;
+      slot[half * 128 + row] = pmax;
+      named_bar_sync(1 + quarter, 64);
+      const float rmax = fmaxf(pmax, slot[(half ^ 1) * 128 + row]);
+
       const float m_new = fmaxf(m_true, rmax);
       const bool upd = (m_new > m_ref) && (m_ref == kNegInf || (m_new - m_ref) * c > 8.0f);
       const float alpha = upd ? ex2((m_ref - m_new) * c) : 1.0f;
       const bool need = upd && (it > 0) && (m_ref != kNegInf);
       if (__any_sync(0xffffffffu, need)) {
-        // rescale O: PV(it-1) must be complete first
-        if (!mbar_wait(bar(C::kBarPVDone), (it - 1) & 1, abort_flag)) { ok = false; break; }
+        // rescale this half of O: PV(it-1) must be complete first
+        if (ok) ok = mbar_wait(bar(C::kBarPVDone), (it - 1) & 1, abort_flag);
         tc_fence_after();
         uint32_t r[32];
 #pragma unroll
-        for (int ch = 0; ch < D / 32; ++ch) {
-          const uint32_t oc = tmem + lane_off + C::kColO + ch * 32;
-          tmem_ld32_wait(oc, r);
+        for (int ch = 0; ch < kHalfD / 32; ++ch) {
+          tmem_ld32_wait(o_col + ch * 32, r);
 #pragma unroll
           for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(__uint_as_float(r[x]) * alpha);
-          tmem_st32(oc, r);
+          tmem_st32(o_col + ch * 32, r);
         }
         tmem_st_wait();
       }
@@ -346,32 +374,30 @@ __global__ void __launch_bounds__(192, 1) attn_dense_kernel(const __grid_constan
       }
       m_true = m_new;
       const float mc = (m_ref == kNegInf) ? 0.f : m_ref * c;
-      uint32_t pk[64];
+      uint32_t pk[32];
       float lsum = 0.f;
 #pragma unroll
-      for (int x = 0; x < 64; ++x) {
+      for (int x = 0; x < 32; ++x) {
         const float p0 = ex2(fmaf(sv[2 * x], c, -mc));
         const float p1 = ex2(fmaf(sv[2 * x + 1], c, -mc));
         lsum += p0 + p1;
         pk[x] = pack_bf16x2(p0, p1);
       }
       l += lsum;
-      {
-        const uint32_t pcol = tmem + lane_off + (bi ? C::kColP1 : C::kColP0);
-        uint32_t r[32];
-#pragma unroll
-        for (int x = 0; x < 32; ++x) r[x] = pk[x];
-        tmem_st32(pcol, r);
-#pragma unroll
-        for (int x = 0; x < 32; ++x) r[x] = pk[32 + x];
-        tmem_st32(pcol + 32, r);
-        tmem_st_wait();
-      }
+      tmem_st32(tmem + lane_off + (bi ? C::kColP1 : C::kColP0) + half * 32, pk);
+      tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar(C::kBarPFull + bi));
     }
 
     // ------------------------------------------------------------ epilogue
+    // total row sum: exchange the two halves' partial sums (slot n&1 was last read at n-2)
+    {
+      float* slot = xch + (n & 1) * 256;
+      slot[half * 128 + row] = l;
+      named_bar_sync(1 + quarter, 64);
+      l += slot[(half ^ 1) * 128 + row];
+    }
     const bool row_valid = i_loc < w.sq;
     bool have_o = ok && n > 0;
     if (have_o) {
@@ -384,13 +410,13 @@ __global__ void __launch_bounds__(192, 1) attn_dense_kernel(const __grid_constan
     if (row_valid) {
       const int64_t orow_idx = p.tnd ? (w.tok0 + i_loc) : i_loc;
       orow = p.out + (p.tnd ? 0 : (int64_t)w.b * p.o_batch_stride) + (int64_t)w.h * p.o_head_stride +
-             orow_idx * p.o_row_stride;
+             orow_idx * p.o_row_stride + half * kHalfD;
     }
 #pragma unroll
-    for (int ch = 0; ch < D / 32; ++ch) {
+    for (int ch = 0; ch < kHalfD / 32; ++ch) {
       uint32_t r[32];
       if (have_o) {
-        tmem_ld32_wait(tmem + lane_off + C::kColO + ch * 32, r);
+        tmem_ld32_wait(o_col + ch * 32, r);
       } else {
 #pragma unroll
         for (int x = 0; x < 32; ++x) r[x] = 0u;
@@ -408,7 +434,7 @@ __global__ void __launch_bounds__(192, 1) attn_dense_kernel(const __grid_constan
         }
       }
     }
-    if (row_valid && (p.softmax_max || p.softmax_sum)) {
+    if (half == 0 && row_valid && (p.softmax_max || p.softmax_sum)) {
       const int64_t sidx = p.tnd ? ((int64_t)w.h * p.stat_head_stride + w.tok0 + i_loc)
                                  : ((int64_t)w.b * p.stat_batch_stride + (int64_t)w.h * p.stat_head_stride + i_loc);
       const bool live = (m_true != kNegInf) && (l > 0.f);

@@ -7,17 +7,22 @@
 // block-sparse mask are computed (section "背景介绍"; block_sparse_mask and
 // block_shape=[128,128] in section "MindIE SD调用方式").
 //
-// One CTA per (batch, head, 128-row query block).  The CTA first compacts its row of
-// the block mask into a list of kept key blocks in shared memory (ascending order),
-// then runs the same warp-specialised pipeline as the dense kernel:
+// One CTA per (batch, head, 128-row query block).  Warp 0 first compacts the CTA's row
+// of the block mask into the ascending list of kept key blocks in shared memory, with
+// each block's dequantisation constant s_q * s_k * scale * log2(e).  Then:
 //   warp 0      TMA producer (Q once; K and V tiles of kept blocks, 3-stage rings)
 //   warp 1      TMEM owner + MMA issuer: S = Q8 K8ᵀ (kind::i8, s32 in TMEM);
 //               O += P8 V8 (kind::f8f6f4, A = P8 from TMEM, B = V8 MN-major) and
 //               L += P8 · 1 (N = 16 ones matrix), so L is exactly Σ p8.
-//   warps 2..5  dequant (exact s32 -> f32, times s_q s_k scale log2 e), online softmax
-//               with the reference max updated at every block (the FP8 rounding of P
-//               depends on it), P -> E4M3 into TMEM, epilogue O * v_scale / L -> bf16.
+//   warps 2..9  softmax: query row 32*(warp%4)+lane; warps 2..5 own key columns [0,64),
+//               warps 6..9 [64,128), exchanging partial row maxima through shared
+//               memory.  Exact s32 -> f32 by the 2^23+2^22 magic add, online softmax with
+//               the reference max updated at every block (the FP8 rounding of P depends
+//               on it), P -> E4M3 into TMEM, epilogue O * v_scale / L -> bf16.
 // TMEM columns: S0 [0,128) S1 [128,256) O [256,384) L [384,400) P0 [448,480) P1 [480,512).
+//
+// CTA order: query heads in groups whose K8/V8 fit in about 48 MB of L2, query blocks
+// in order, heads fastest inside a group.
 #pragma once
 
 #include <cstdint>
@@ -42,6 +47,8 @@ struct QbsaParams {
   float* softmax_max;     // [B, Nq, Sq] or nullptr
   float* softmax_sum;
   int B, Nq, Nkv, Sq, Skv, group, nqb, nkb;
+  int n_rank;             // B * nqb
+  int head_grp;           // query heads per L2 group
   float scale_log2;       // scale * log2(e)
 };
 
@@ -53,8 +60,10 @@ struct QbsaCfg {
   static constexpr int kKOff = kQOff + kTileBytes;
   static constexpr int kVOff = kKOff + kStages * kTileBytes;
   static constexpr int kOnesOff = kVOff + kStages * kTileBytes;  // 16 x 128 bytes of E4M3 1.0
-  static constexpr int kListOff = kOnesOff + 2048;                // uint16 kept-block list
-  static constexpr int kBarOff = kListOff + kQbsaMaxKBlocks * 2;
+  static constexpr int kCOff = kOnesOff + 2048;                   // float dequant constant per kept block
+  static constexpr int kListOff = kCOff + kQbsaMaxKBlocks * 4;    // uint16 kept-block list
+  static constexpr int kXOff = kListOff + kQbsaMaxKBlocks * 2;    // int row-max exchange [2][2][128]
+  static constexpr int kBarOff = kXOff + 2 * 2 * 128 * 4;
   static constexpr int kBarQFull = 0;
   static constexpr int kBarKFull = 1;
   static constexpr int kBarKEmpty = kBarKFull + kStages;
@@ -70,7 +79,8 @@ struct QbsaCfg {
   static constexpr int kSmemBytes = kMiscOff + 16 + 1024;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256, kColL = 384, kColP0 = 448, kColP1 = 480;
-  static constexpr int kThreads = 192;
+  static constexpr int kThreads = 320;
+  static constexpr int kSoftmaxThreads = 256;
 };
 
 // Compact one row of the block mask (n_kb bytes, 1 = keep) into ascending indices.
@@ -87,7 +97,16 @@ __device__ __forceinline__ int compact_mask_row(const uint8_t* row, int n_kb, ui
   return count;
 }
 
-__global__ void __launch_bounds__(192, 1) attn_qbsa_kernel(const __grid_constant__ QbsaParams p) {
+__device__ __forceinline__ void qbsa_named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// Exact int32 -> float32 for |t| < 2^22 on the FMA pipe: the bits of 2^23 + 2^22 + t.
+__device__ __forceinline__ float s32_to_f32_exact(int32_t t) {
+  return __int_as_float(t + 0x4B400000) - 12582912.0f;
+}
+
+__global__ void __launch_bounds__(320, 1) attn_qbsa_kernel(const __grid_constant__ QbsaParams p) {
   using C = QbsaCfg;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
@@ -102,15 +121,28 @@ __global__ void __launch_bounds__(192, 1) attn_qbsa_kernel(const __grid_constant
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
   int* count_slot = reinterpret_cast<int*>(smem + C::kMiscOff + 8);
   uint16_t* list = reinterpret_cast<uint16_t*>(smem + C::kListOff);
+  float* cst_list = reinterpret_cast<float*>(smem + C::kCOff);
+  int32_t* xch = reinterpret_cast<int32_t*>(smem + C::kXOff);
 
-  const int h = static_cast<int>(blockIdx.x % p.Nq);
-  const int qb = static_cast<int>((blockIdx.x / p.Nq) % p.nqb);
-  const int b = static_cast<int>(blockIdx.x / p.Nq / p.nqb);
+  // head groups (L2 reuse of K/V), query blocks in order, heads fastest inside a group
+  const int64_t per_group = (int64_t)p.head_grp * p.n_rank;
+  const int grp = static_cast<int>(blockIdx.x / per_group);
+  const int h0 = grp * p.head_grp;
+  const int hcount = min(p.head_grp, p.Nq - h0);
+  const int off = static_cast<int>(blockIdx.x - grp * per_group);
+  const int r = off / hcount;
+  const int h = h0 + off % hcount;
+  const int qb = r % p.nqb;
+  const int b = r / p.nqb;
   const int g = h / p.group;
 
   if (warp == 0) {
     const uint8_t* mrow = p.block_mask + (((int64_t)b * p.Nq + h) * p.nqb + qb) * p.nkb;
     const int cnt = compact_mask_row(mrow, p.nkb, list, lane);
+    __syncwarp();
+    const float sq = p.q_scale[((int64_t)b * p.Nq + h) * p.nqb + qb];
+    const float* ks = p.k_scale + ((int64_t)b * p.Nkv + g) * p.nkb;
+    for (int i = lane; i < cnt; i += 32) cst_list[i] = (sq * ks[list[i]]) * p.scale_log2;
     if (lane == 0) {
       *count_slot = cnt;
       *abort_flag = 0;
@@ -123,8 +155,8 @@ __global__ void __launch_bounds__(192, 1) attn_qbsa_kernel(const __grid_constant
       }
       for (int b2 = 0; b2 < 2; ++b2) {
         mbar_init(bar(C::kBarSFull + b2), 1);
-        mbar_init(bar(C::kBarSFree + b2), 128);
-        mbar_init(bar(C::kBarPFull + b2), 128);
+        mbar_init(bar(C::kBarSFree + b2), C::kSoftmaxThreads);
+        mbar_init(bar(C::kBarPFull + b2), C::kSoftmaxThreads);
       }
       mbar_init(bar(C::kBarPVDone), 1);
       mbar_init(bar(C::kBarOFinal), 1);
@@ -218,28 +250,30 @@ __global__ void __launch_bounds__(192, 1) attn_qbsa_kernel(const __grid_constant
   } else {
     // ---------------------------------------------------------------- softmax warps
     const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;  // 0: key columns [0,64), 1: [64,128)
     const int row = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const int64_t i_glob = (int64_t)qb * kTile + row;
     const float kNegInf = -__int_as_float(0x7f800000);
-    const float sq_scale = p.q_scale[((int64_t)b * p.Nq + h) * p.nqb + qb];
-    const float* ks_row = p.k_scale + ((int64_t)b * p.Nkv + g) * p.nkb;
+    const uint32_t o_col = tmem + lane_off + C::kColO + half * 64;
+    const uint32_t l_col = tmem + lane_off + C::kColL;
 
     float m = kNegInf;  // running max, log2 domain
     bool ok = true;
     for (int it = 0; it < n; ++it) {
       const int kb = list[it];
       const int bi = it & 1;
-      const float cst = (sq_scale * ks_row[kb]) * p.scale_log2;
-      const int valid = min(kTile, p.Skv - kb * kTile);  // columns inside S_kv
-      if (!mbar_wait(bar(C::kBarSFull + bi), (it >> 1) & 1, abort_flag)) { ok = false; break; }
+      const float cst = cst_list[it];
+      const int valid = min(kTile, p.Skv - kb * kTile) - half * 64;  // valid columns of this half
+      // never leave the loop early (the paired warp waits on named barriers below)
+      if (ok) ok = mbar_wait(bar(C::kBarSFull + bi), (it >> 1) & 1, abort_flag);
       tc_fence_after();
-      int32_t sv[128];
+      int32_t sv[64];
       {
         uint32_t r[32];
-        const uint32_t scol = tmem + lane_off + (bi ? C::kColS1 : C::kColS0);
+        const uint32_t scol = tmem + lane_off + (bi ? C::kColS1 : C::kColS0) + half * 64;
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
+        for (int ch = 0; ch < 2; ++ch) {
           tmem_ld32_wait(scol + ch * 32, r);
 #pragma unroll
           for (int x = 0; x < 32; ++x) sv[ch * 32 + x] = static_cast<int32_t>(r[x]);
@@ -248,49 +282,59 @@ __global__ void __launch_bounds__(192, 1) attn_qbsa_kernel(const __grid_constant
       tc_fence_before();
       mbar_arrive(bar(C::kBarSFree + bi));
 
-      if (valid < kTile) {
+      if (valid < 64) {
 #pragma unroll
-        for (int x = 0; x < 128; ++x)
+        for (int x = 0; x < 64; ++x)
           if (x >= valid) sv[x] = INT32_MIN;
       }
-      int32_t tmax = sv[0];
+      int32_t pmax = max(sv[0], sv[1]);
 #pragma unroll
-      for (int x = 1; x < 128; ++x) tmax = max(tmax, sv[x]);
-      const float m_blk = static_cast<float>(tmax) * cst;
+      for (int x = 2; x < 64; x += 2) pmax = max(pmax, max(sv[x], sv[x + 1]));
+      int32_t* slot = xch + (it & 1) * 256;
+      slot[half * 128 + row] = pmax;
+      qbsa_named_bar_sync(1 + quarter, 64);
+      const int32_t tmax = max(pmax, slot[(half ^ 1) * 128 + row]);
+
+      const float m_blk = s32_to_f32_exact(tmax) * cst;
       const float m_new = fmaxf(m, m_blk);
       const bool upd = m_new > m;
       const float alpha = (m == kNegInf) ? 0.f : ex2(m - m_new);
       const bool need = upd && (it > 0) && (m != kNegInf);
       if (__any_sync(0xffffffffu, need)) {
-        if (!mbar_wait(bar(C::kBarPVDone), (it - 1) & 1, abort_flag)) { ok = false; break; }
+        if (ok) ok = mbar_wait(bar(C::kBarPVDone), (it - 1) & 1, abort_flag);
         tc_fence_after();
         const float a = upd ? alpha : 1.0f;
         uint32_t r[32];
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          const uint32_t oc = tmem + lane_off + C::kColO + ch * 32;
-          tmem_ld32_wait(oc, r);
+        for (int ch = 0; ch < 2; ++ch) {
+          tmem_ld32_wait(o_col + ch * 32, r);
 #pragma unroll
           for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(__uint_as_float(r[x]) * a);
-          tmem_st32(oc, r);
+          tmem_st32(o_col + ch * 32, r);
         }
-        const uint32_t lc = tmem + lane_off + C::kColL;
-        tmem_st1(lc, __float_as_uint(__uint_as_float(tmem_ld1_wait(lc)) * a));
+        if (half == 0) tmem_st1(l_col, __float_as_uint(__uint_as_float(tmem_ld1_wait(l_col)) * a));
         tmem_st_wait();
       }
       m = m_new;
-      uint32_t pk[32];
+      uint32_t pk[16];
 #pragma unroll
-      for (int x = 0; x < 32; ++x) {
+      for (int x = 0; x < 16; ++x) {
         float pv[4];
 #pragma unroll
-        for (int y = 0; y < 4; ++y) {
-          const int32_t t = sv[4 * x + y];
-          pv[y] = (t == INT32_MIN) ? 0.f : ex2(fmaf(static_cast<float>(t), cst, -m));
-        }
+        for (int y = 0; y < 4; ++y) pv[y] = ex2(fmaf(s32_to_f32_exact(sv[4 * x + y]), cst, -m));
         pk[x] = pack_e4m3x4(pv[0], pv[1], pv[2], pv[3]);
       }
-      tmem_st32(tmem + lane_off + (bi ? C::kColP1 : C::kColP0), pk);
+      if (valid < 64) {  // tail block: masked keys get p = 0
+#pragma unroll
+        for (int x = 0; x < 16; ++x) {
+          uint32_t keep = 0;
+#pragma unroll
+          for (int y = 0; y < 4; ++y)
+            if (4 * x + y < valid) keep |= 0xFFu << (8 * y);
+          pk[x] &= keep;
+        }
+      }
+      tmem_st16(tmem + lane_off + (bi ? C::kColP1 : C::kColP0) + half * 16, pk);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar(C::kBarPFull + bi));
@@ -305,15 +349,15 @@ __global__ void __launch_bounds__(192, 1) attn_qbsa_kernel(const __grid_constant
       tc_fence_after();
     }
     float l = 0.f;
-    if (have_o) l = __uint_as_float(tmem_ld1_wait(tmem + lane_off + C::kColL));
+    if (have_o) l = __uint_as_float(tmem_ld1_wait(l_col));
     const float inv_l = (l > 0.f) ? 1.0f / l : 0.f;
-    const float* vsc = p.v_scale + ((int64_t)b * p.Nkv + g) * 128;
-    __nv_bfloat16* orow = p.out + (((int64_t)b * p.Nq + h) * p.Sq + i_glob) * 128;
+    const float* vsc = p.v_scale + ((int64_t)b * p.Nkv + g) * 128 + half * 64;
+    __nv_bfloat16* orow = p.out + (((int64_t)b * p.Nq + h) * p.Sq + i_glob) * 128 + half * 64;
 #pragma unroll
-    for (int ch = 0; ch < 4; ++ch) {
+    for (int ch = 0; ch < 2; ++ch) {
       uint32_t r[32];
       if (have_o) {
-        tmem_ld32_wait(tmem + lane_off + C::kColO + ch * 32, r);
+        tmem_ld32_wait(o_col + ch * 32, r);
       } else {
 #pragma unroll
         for (int x = 0; x < 32; ++x) r[x] = 0u;
@@ -334,7 +378,7 @@ __global__ void __launch_bounds__(192, 1) attn_qbsa_kernel(const __grid_constant
         }
       }
     }
-    if (row_valid) {
+    if (half == 0 && row_valid) {
       const int64_t sidx = ((int64_t)b * p.Nq + h) * p.Sq + i_glob;
       const bool live = l > 0.f;
       if (p.softmax_max) p.softmax_max[sidx] = live ? m * 0.6931471805599453f : kNegInf;

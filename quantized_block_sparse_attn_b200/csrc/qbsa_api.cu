@@ -80,6 +80,14 @@ qbsa_status make_map(CUtensorMap* map, CUtensorMapDataType dt, const void* ptr, 
   return QBSA_OK;
 }
 
+// Query heads per CTA group so that the group's K/V (kv_bytes_per_qhead each) stay in
+// roughly 48 MB of the 126 MB L2 while the group's CTAs run.
+int head_group(double kv_bytes_per_qhead, int n_heads) {
+  const double budget = 48.0 * 1024 * 1024;
+  int g = static_cast<int>(budget / std::max(kv_bytes_per_qhead, 1.0));
+  return std::max(1, std::min(g, n_heads));
+}
+
 template <typename K>
 qbsa_status set_smem(K kernel, int bytes) {
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
@@ -267,6 +275,9 @@ qbsa_status attn_fwd(const void* q, const void* k, const void* v, int B, int Nq,
   const int64_t n_work = n_rank * Nq;
   if (n_work == 0) return QBSA_OK;
   if (n_work > 0x7fffffffLL) return fail(QBSA_ERR_UNSUPPORTED, "too many query tiles (%lld)", (long long)n_work);
+  prm.n_rank = static_cast<int>(n_rank);
+  // K/V bytes of one query head: one kv head (all batches; all sequences for TND) over the group
+  prm.head_grp = head_group(static_cast<double>(std::max(Skv, 1)) * D * 2 * 2 * (tnd ? 1 : B) / prm.group, Nq);
 
   qbsa_status st;
   if ((st = make_map(&prm.tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, qd, qs, 64)) != QBSA_OK) return st;
@@ -318,6 +329,9 @@ qbsa_status qbsa_fwd(const int8_t* q_i8, const int8_t* k_i8, const float* q_bloc
   prm.nqb = nqb;
   prm.nkb = nkb;
   prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.n_rank = B * nqb;
+  // K8 + V8 bytes of one query head: one kv head over all batches, shared by the group
+  prm.head_grp = head_group(static_cast<double>(std::max(Skv, 1)) * 128 * 2 * B / prm.group, Nq);
   const int64_t n_work = (int64_t)B * nqb * Nq;
   if (n_work > 0x7fffffffLL) return fail(QBSA_ERR_UNSUPPORTED, "too many query blocks");
   if (Skv == 0) {
