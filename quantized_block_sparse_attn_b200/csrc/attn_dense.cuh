@@ -310,14 +310,10 @@ __global__ void __launch_bounds__(320, 1) attn_dense_kernel(const __grid_constan
       tc_fence_after();
       float sv[64];
       {
-        uint32_t r[32];
-        const uint32_t scol = tmem + lane_off + (bi ? C::kColS1 : C::kColS0) + half * 64;
+        uint32_t r[64];
+        tmem_ld64_wait(tmem + lane_off + (bi ? C::kColS1 : C::kColS0) + half * 64, r);
 #pragma unroll
-        for (int ch = 0; ch < 2; ++ch) {
-          tmem_ld32_wait(scol + ch * 32, r);
-#pragma unroll
-          for (int x = 0; x < 32; ++x) sv[ch * 32 + x] = __uint_as_float(r[x]);
-        }
+        for (int x = 0; x < 64; ++x) sv[x] = __uint_as_float(r[x]);
       }
       tc_fence_before();
       mbar_arrive(bar(C::kBarSFree + bi));
@@ -341,9 +337,7 @@ __global__ void __launch_bounds__(320, 1) attn_dense_kernel(const __grid_constan
           sv[x] = keep ? v : kNegInf;
         }
       }
-      float pmax = sv[0];
-#pragma unroll
-      for (int x = 1; x < 64; ++x) pmax = fmaxf(pmax, sv[x]);
+      const float pmax = max64(sv);
       // combine the two halves of the row
       float* slot = xch + (it & 1) * 256;
       slot[half * 128 + row] = pmax;
@@ -375,15 +369,15 @@ __global__ void __launch_bounds__(320, 1) attn_dense_kernel(const __grid_constan
       m_true = m_new;
       const float mc = (m_ref == kNegInf) ? 0.f : m_ref * c;
       uint32_t pk[32];
-      float lsum = 0.f;
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};  // independent partial sums (short dependency chains)
 #pragma unroll
       for (int x = 0; x < 32; ++x) {
         const float p0 = ex2(fmaf(sv[2 * x], c, -mc));
         const float p1 = ex2(fmaf(sv[2 * x + 1], c, -mc));
-        lsum += p0 + p1;
+        ls[x & 3] += p0 + p1;
         pk[x] = pack_bf16x2(p0, p1);
       }
-      l += lsum;
+      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
       tmem_st32(tmem + lane_off + (bi ? C::kColP1 : C::kColP0) + half * 32, pk);
       tmem_st_wait();
       tc_fence_before();

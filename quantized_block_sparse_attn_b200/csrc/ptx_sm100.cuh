@@ -228,6 +228,20 @@ __device__ __forceinline__ void tmem_ld32_wait(uint32_t taddr, uint32_t (&r)[32]
       : "memory");
 }
 
+// Load 64 consecutive 32-bit columns of this warp's 32 lanes in one round trip.
+__device__ __forceinline__ void tmem_ld64_wait(uint32_t taddr, uint32_t (&r)[64]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,"
+      "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+      "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : QBSA_R8(0), QBSA_R8(8), QBSA_R8(16), QBSA_R8(24), QBSA_R8(32), QBSA_R8(40), QBSA_R8(48), QBSA_R8(56)
+      : "r"(taddr)
+      : "memory");
+}
+
 // Load one 32-bit column (lane = thread) and wait.
 __device__ __forceinline__ uint32_t tmem_ld1_wait(uint32_t taddr) {
   uint32_t v;
@@ -273,6 +287,25 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Three-input maximum (one instruction on sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Maximum of 64 values as a depth-4 tree of three-input maxima (32 instructions).
+__device__ __forceinline__ float max64(const float (&v)[64]) {
+  float a[22], b[8];
+#pragma unroll
+  for (int i = 0; i < 21; ++i) a[i] = fmax3(v[3 * i], v[3 * i + 1], v[3 * i + 2]);
+  a[21] = v[63];
+#pragma unroll
+  for (int i = 0; i < 7; ++i) b[i] = fmax3(a[3 * i], a[3 * i + 1], a[3 * i + 2]);
+  b[7] = a[21];
+  return fmax3(fmax3(b[0], b[1], b[2]), fmax3(b[3], b[4], b[5]), fmaxf(b[6], b[7]));
 }
 
 // Two f32 -> packed bf16x2 (lo in bits [0,16)), round to nearest even.
