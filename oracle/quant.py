@@ -5,7 +5,10 @@ Source: EagleQBSA article, "昇腾MindIE SD高性能量化稀疏联合注意力E
 * Section "EagleQBSA量化叠加稀疏方案设计" and Fig 2.1: Q and K are quantised to
   INT8, symmetric and linear, one scale per 128-token block of the sequence axis;
   V is quantised to FP8 E4M3 with one scale per channel (head-dim column) covering
-  the whole sequence; the attention probabilities P are rounded to FP8 before P·V.
+  the whole sequence; the attention map P is rounded to FP8 before P·V.
+* Section "昇腾亲和的量化叠加稀疏Attention算子优化": P is held in floating point
+  (FP16 there) and converted to FP8; the conversion rounds each weight's mantissa at
+  its own binary exponent.
 * Section "MindIE SD调用方式": the operator receives the INT8 query/key, the E4M3
   value bytes, query_scale / key_scale / value_scale, a block_sparse_mask with
   block_shape [128, 128], scale_value (the softmax scale, 128^-0.5 in the example)
@@ -21,32 +24,46 @@ Readings where the article is silent (each also listed in the design notes):
 * Shapes: query_scale [B, N_q, ceil(S_q/128)], key_scale [B, N_kv, ceil(S_kv/128)],
   value_scale [B, N_kv, D]; block_sparse_mask uint8 [B, N_q, ceil(S_q/128),
   ceil(S_kv/128)] with 1 = compute the block.
-* Score: s = t * s_q * s_k * scale, t the exact integer dot product of the INT8 rows.
-* Kept blocks are visited in ascending key order; the softmax runs online, one
-  128-key block per step: m_new = max(m, rowmax s); p = exp(s - m_new) held in
-  float32 (the precision in which the FP8 rounding decision is taken) and rounded to
-  E4M3 (nearest even); l = l * exp(m - m_new) + Σ p8 (the sum of the ROUNDED
-  weights); acc = acc * exp(m - m_new) + p8 · v8.
-* Output O[:, c] = acc[:, c] / l * v_scale[c]; softmax_max = final m; softmax_sum =
-  final l.  A row with no kept block returns O = 0, max = -inf, sum = 0.
+* Score: s = t * s_q * s_k * scale, t the exact integer dot product of the INT8 rows;
+  z = s * log2(e) is the same score in base-2 units.
+* Kept blocks are visited in ascending key order, one 128-key block per step.  The
+  weights are taken against a power-of-two reference R (an integer in log2 units)
+  that follows the running max m of z lazily: at a block, m = max(m, rowmax z); if R
+  is unset or m > R + 8, R = ceil(m) and the accumulated l and acc are multiplied by
+  the exact power of two 2^(R_old - R).  Then p = 2^(z - R) <= 2^8 (below E4M3's 448).
+  The article fixes neither the reference nor when it moves.  A power-of-two
+  reference makes the rescaling exact, and E4M3 rounding commutes with powers of two,
+  so the codes equal those against the final max except for weights in E4M3's
+  subnormal range (below 2^-6 of the reference).
+* p is held in float32 (the precision in which the FP8 decision is taken) and
+  rounded to E4M3 (nearest even): p8 = E4M3(p).  l = Σ p8 (the sum of the ROUNDED
+  weights, so constant V returns V exactly); O[:, c] = acc[:, c] / l · v_scale[c]
+  with acc = Σ p8 · v8.
+* softmax_max = final m in the natural-log domain (max s) and softmax_sum = l · 2^(R - m):
+  the sum of the rounded weights expressed against the true row maximum.
+* A row with no kept block returns O = 0, softmax_max = -inf, softmax_sum = 0.
 
 Parity pins (tests): the quantiser codes meet the rounding bound |x - q s| <= s/2 and
 hit ±127 at the block maximum; the E4M3 codec matches the OCP definition on every
 code and torch's float8_e4m3fn cast on finite inputs; with P rounding switched off the
-online recurrence equals the direct softmax over the kept keys; q = 0 gives p8 = 1,
-softmax_sum = 128 x kept blocks and O = the mean of the dequantised V; constant V
-returns V; a pure-Python loop version agrees on tiny inputs; masked-out blocks have
-no influence.  The article prints no quantisation error figure ("parity unpinned"
-for the article's own error level; only VBench scores are given, out of scope).
+result equals the dense oracle restricted to the kept blocks; q = 0 gives p8 = 1,
+softmax_sum = the kept-key count and O = the mean of the dequantised V; constant V
+returns V; a pure-Python loop version agrees on tiny inputs; masked-out blocks have no
+influence.  The article prints no quantisation error figure ("parity unpinned" for
+the article's own error level; only VBench scores are given, out of scope).
 """
 
 from __future__ import annotations
+
+import math
 
 import numpy as np
 
 from .formats import bf16_to_f64, e4m3_encode, e4m3_decode
 
 BLK = 128
+LOG2E = 1.0 / math.log(2.0)
+REF_SLACK = 8  # the reference is re-set once the running max exceeds it by more than 8 (log2 units)
 
 
 # --------------------------------------------------------------------------------------
@@ -91,34 +108,37 @@ def quantize_v_per_channel(v):
 # the forward
 # --------------------------------------------------------------------------------------
 
-def _head_forward(q8, k8, qs, ks, v8f, vs, mask_rows, scale, skv, qbs, round_p=True):
+def _head_forward(q8, k8, qs, ks, v8f, vs, mask_rows, scale, qbs, round_p=True):
     """One (b, h): q8 [Sq, D] int8, k8 [Skv, D], v8f [Skv, D] decoded E4M3, per-block scales."""
-    D = v8f.shape[1]
+    skv, D = k8.shape[0], v8f.shape[1]
     outs, mxs, sms = [], [], []
     for qb in qbs:
         r0, r1 = qb * BLK, min(q8.shape[0], (qb + 1) * BLK)
         rows = r1 - r0
-        m = np.full(rows, -np.inf)
+        qi = q8[r0:r1].astype(np.int64)
+        m = np.full(rows, -np.inf)     # running max of z
+        ref = np.full(rows, -np.inf)   # power-of-two reference R (an integer)
         l = np.zeros(rows)
         acc = np.zeros((rows, D))
-        qi = q8[r0:r1].astype(np.int64)
-        for kb in np.nonzero(mask_rows[qb])[0]:
+        for kb in np.nonzero(mask_rows[qb])[0]:                               # ascending
             c0, c1 = kb * BLK, min(skv, (kb + 1) * BLK)
-            t = qi @ k8[c0:c1].astype(np.int64).T                     # exact integers
-            s = t.astype(np.float64) * (float(qs[qb]) * float(ks[kb]) * scale)
-            m_new = np.maximum(m, s.max(axis=1))
-            alpha = np.where(np.isfinite(m), np.exp(m - m_new), 0.0)
-            p = np.exp(s - m_new[:, None])
+            t = qi @ k8[c0:c1].astype(np.int64).T                              # exact integers
+            z = t.astype(np.float64) * (float(qs[qb]) * float(ks[kb]) * scale) * LOG2E
+            m = np.maximum(m, z.max(axis=1))
+            upd = np.isneginf(ref) | (m > ref + REF_SLACK)
+            new_ref = np.where(upd, np.ceil(m), ref)
+            unset = np.isneginf(ref)
+            alpha = np.where(unset, 0.0, np.exp2(np.where(unset, 0.0, ref) - new_ref))  # exact powers of two
+            l, acc, ref = l * alpha, acc * alpha[:, None], new_ref
+            p = np.exp2(z - ref[:, None])
             if round_p:
                 p = e4m3_decode(e4m3_encode(p.astype(np.float32)))
-            l = l * alpha + p.sum(axis=1)
-            acc = acc * alpha[:, None] + p @ v8f[c0:c1]
-            m = m_new
+            l = l + p.sum(axis=1)
+            acc = acc + p @ v8f[c0:c1]
         live = l > 0
-        o = np.where(live[:, None], acc / np.where(live, l, 1.0)[:, None], 0.0) * vs[None, :]
-        outs.append(o)
-        mxs.append(m)
-        sms.append(l)
+        outs.append(np.where(live[:, None], acc / np.where(live, l, 1.0)[:, None], 0.0) * vs[None, :])
+        mxs.append(m / LOG2E)
+        sms.append(np.where(live, l * np.exp2(np.where(live, ref - m, 0.0)), 0.0))
     return outs, mxs, sms
 
 
@@ -137,7 +157,7 @@ def qbsa_forward(q8, k8, q_scale, k_scale, v8, v_scale, block_mask, scale: float
     q8 = np.asarray(q8)
     k8 = np.asarray(k8)
     B, Nq, Sq, D = q8.shape
-    Nkv, Skv = k8.shape[1], k8.shape[2]
+    Nkv = k8.shape[1]
     group = Nq // Nkv
     nqb = -(-Sq // BLK)
     out = np.full((B, Nq, Sq, D), np.nan)
@@ -150,9 +170,9 @@ def qbsa_forward(q8, k8, q_scale, k_scale, v8, v_scale, block_mask, scale: float
         g = h // group
         if (b, g) not in v8f_cache:
             v8f_cache[(b, g)] = e4m3_decode(v8[b, g])
-        o, mx, sm = _head_forward(q8[b, h], k8[b, g], q_scale[b, h], k_scale[b, g],
-                                  v8f_cache[(b, g)], np.asarray(v_scale[b, g], dtype=np.float64),
-                                  block_mask[b, h], scale, Skv, qbs, round_p)
+        o, mx, sm = _head_forward(q8[b, h], k8[b, g], q_scale[b, h], k_scale[b, g], v8f_cache[(b, g)],
+                                  np.asarray(v_scale[b, g], dtype=np.float64), block_mask[b, h], scale, qbs,
+                                  round_p)
         for qb, oo, mm, ss in zip(qbs, o, mx, sm):
             r0, r1 = qb * BLK, min(Sq, (qb + 1) * BLK)
             out[b, h, r0:r1] = oo
@@ -162,8 +182,7 @@ def qbsa_forward(q8, k8, q_scale, k_scale, v8, v_scale, block_mask, scale: float
 
 
 def qbsa_forward_loops(q8, k8, q_scale, k_scale, v8, v_scale, block_mask, scale: float):
-    """The same forward with explicit Python loops over rows, blocks and keys (tiny inputs)."""
-    import math
+    """The same forward with explicit Python loops over rows and keys (tiny inputs)."""
     q8 = np.asarray(q8)
     k8 = np.asarray(k8)
     B, Nq, Sq, D = q8.shape
@@ -177,30 +196,32 @@ def qbsa_forward_loops(q8, k8, q_scale, k_scale, v8, v_scale, block_mask, scale:
             g = h // group
             for i in range(Sq):
                 qb = i // BLK
-                m, l = -math.inf, 0.0
+                m, ref, l = -math.inf, -math.inf, 0.0
                 acc = [0.0] * D
                 for kb in range(block_mask.shape[3]):
                     if not block_mask[b, h, qb, kb]:
                         continue
                     cols = range(kb * BLK, min(Skv, (kb + 1) * BLK))
-                    s = []
+                    z = []
                     for j in cols:
                         t = sum(int(q8[b, h, i, c]) * int(k8[b, g, j, c]) for c in range(D))
-                        s.append(t * (float(q_scale[b, h, qb]) * float(k_scale[b, g, kb]) * scale))
-                    m_new = max(m, max(s))
-                    alpha = math.exp(m - m_new) if m != -math.inf else 0.0
-                    l *= alpha
-                    acc = [a * alpha for a in acc]
-                    for j, sj in zip(cols, s):
-                        p = float(e4m3_decode(e4m3_encode(np.float32(math.exp(sj - m_new)))))
+                        z.append(t * (float(q_scale[b, h, qb]) * float(k_scale[b, g, kb]) * scale) * LOG2E)
+                    m = max(m, max(z))
+                    if ref == -math.inf or m > ref + REF_SLACK:
+                        new_ref = math.ceil(m)
+                        alpha = 0.0 if ref == -math.inf else 2.0 ** (ref - new_ref)
+                        l *= alpha
+                        acc = [a * alpha for a in acc]
+                        ref = new_ref
+                    for j, zj in zip(cols, z):
+                        p = float(e4m3_decode(e4m3_encode(np.float32(2.0 ** (zj - ref)))))
                         l += p
                         vrow = e4m3_decode(v8[b, g, j])
                         for c in range(D):
                             acc[c] += p * vrow[c]
-                    m = m_new
                 if l > 0:
                     for c in range(D):
                         out[b, h, i, c] = acc[c] / l * float(v_scale[b, g, c])
-                smax[b, h, i] = m
-                ssum[b, h, i] = l
+                    smax[b, h, i] = m / LOG2E
+                    ssum[b, h, i] = l * 2.0 ** (ref - m)
     return out, smax, ssum

@@ -88,6 +88,28 @@ def test_online_recurrence_without_p_rounding_equals_direct_softmax():
     assert np.allclose(out, _direct_softmax(p, 0.25), rtol=1e-11, atol=1e-12)
 
 
+@pytest.mark.parametrize("seed,D,scale", [(10, 16, 0.5), (11, 64, 0.2), (12, 128, 128 ** -0.5)])
+def test_power_of_two_reference_matches_final_max_up_to_subnormals(seed, D, scale):
+    """The lazily moved power-of-two reference gives the codes of the order-free
+    definition p8 = E4M3(2^(z - ceil(max z))) except where a weight falls in E4M3's
+    subnormal range (below 2^-6) on one side: each such weight moves by at most the
+    subnormal spacing 2^-9 (in units of the final reference), which bounds the output."""
+    from oracle.formats import e4m3_decode, e4m3_encode
+    p = _problem(seed, Nq=1, Nkv=1, Sq=128, Skv=1024, D=D, keep=1.0)
+    got, _, _ = quant.qbsa_forward(p["q8"], p["k8"], p["qs"], p["ks"], p["v8"], p["vs"], p["bm"], scale)
+    q8, k8 = p["q8"][0, 0].astype(np.int64), p["k8"][0, 0].astype(np.int64)
+    ks_col = np.repeat(p["ks"][0, 0].astype(np.float64), 128)
+    z = (q8 @ k8.T) * (float(p["qs"][0, 0, 0]) * ks_col[None, :] * scale) / np.log(2.0)
+    M = np.ceil(z.max(axis=1))
+    w = np.exp2(z - M[:, None])
+    w8 = e4m3_decode(e4m3_encode(w.astype(np.float32)))
+    vdq = e4m3_decode(p["v8"][0, 0]) * p["vs"][0, 0][None, :]
+    two_pass = (w8 @ vdq) / w8.sum(axis=1)[:, None]
+    n_sub = (w < 2.0 ** -6).sum(axis=1)
+    bound = 2 * n_sub * 2.0 ** -9 * np.abs(vdq).max() / w8.sum(axis=1)
+    assert np.all(np.abs(got[0, 0] - two_pass) <= bound[:, None] + 1e-12)
+
+
 def test_loops_equal_vectorised_tiny():
     p = _problem(4, Nq=2, Nkv=1, Sq=140, Skv=200, D=4, keep=1.0)
     a = quant.qbsa_forward(p["q8"], p["k8"], p["qs"], p["ks"], p["v8"], p["vs"], p["bm"], 0.5)
