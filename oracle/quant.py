@@ -138,7 +138,7 @@ def _head_forward(q8, k8, qs, ks, v8f, vs, mask_rows, scale, qbs, round_p=True):
         live = l > 0
         outs.append(np.where(live[:, None], acc / np.where(live, l, 1.0)[:, None], 0.0) * vs[None, :])
         mxs.append(m / LOG2E)
-        sms.append(np.where(live, l * np.exp2(np.where(live, ref - m, 0.0)), 0.0))
+        sms.append(np.where(live, l * np.exp2(np.where(live, ref, 0.0) - np.where(live, m, 0.0)), 0.0))
     return outs, mxs, sms
 
 

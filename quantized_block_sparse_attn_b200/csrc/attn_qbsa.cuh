@@ -16,9 +16,11 @@
 //               L += P8 · 1 (N = 16 ones matrix), so L is exactly Σ p8.
 //   warps 2..9  softmax: query row 32*(warp%4)+lane; warps 2..5 own key columns [0,64),
 //               warps 6..9 [64,128), exchanging partial row maxima through shared
-//               memory.  Exact s32 -> f32 (|dot| < 2^24), online softmax with the
-//               reference max updated at every block (the FP8 rounding of P depends on
-//               it), P -> E4M3 into TMEM, epilogue O * v_scale / L -> bf16.
+//               memory.  Exact s32 -> f32 (|dot| < 2^24), online softmax whose weights
+//               p = 2^(z - R) use a power-of-two reference R re-set to ceil(running max)
+//               only when the max exceeds it by more than 8 (exact power-of-two
+//               rescales of O and L, rare), P -> E4M3 into TMEM, epilogue
+//               O * v_scale / L -> bf16.
 // TMEM columns: S0 [0,128) S1 [128,256) O [256,384) L [384,400) P0 [448,480) P1 [480,512).
 //
 // CTA order: query heads in groups whose K8/V8 fit in about 48 MB of L2, query blocks
@@ -253,7 +255,8 @@ __global__ void __launch_bounds__(320, 1) attn_qbsa_kernel(const __grid_constant
     const uint32_t o_col = tmem + lane_off + C::kColO + half * 64;
     const uint32_t l_col = tmem + lane_off + C::kColL;
 
-    float m = kNegInf;  // running max, log2 domain
+    float m = kNegInf;    // running max, log2 domain
+    float ref = kNegInf;  // power-of-two reference of the FP8 weights (an integer)
     bool ok = true;
     for (int it = 0; it < n; ++it) {
       const int kb = list[it];
@@ -286,14 +289,19 @@ __global__ void __launch_bounds__(320, 1) attn_qbsa_kernel(const __grid_constant
 
       // max(t) * c == max(t * c): multiplication by c > 0 is monotone in float
       const float m_blk = tmax * cst;
-      const float m_new = fmaxf(m, m_blk);
-      const bool upd = m_new > m;
-      const float alpha = (m == kNegInf) ? 0.f : ex2(m - m_new);
-      const bool need = upd && (it > 0) && (m != kNegInf);
+      m = fmaxf(m, m_blk);
+      // power-of-two reference: re-set to ceil(m) once m exceeds it by more than 8, so
+      // p <= 2^8 stays below E4M3's 448 and every rescale is an exact power of two
+      const bool upd = (ref == kNegInf) || (m > ref + 8.0f);
+      const float new_ref = upd ? ceilf(m) : ref;
+      const bool need = upd && (ref != kNegInf);
+      // 2^(ref - new_ref) built from its exponent bits (exact; flush below 2^-126)
+      const int dexp = need ? static_cast<int>(ref - new_ref) : 0;
+      const float a = (dexp < -126) ? 0.f : __int_as_float((127 + dexp) << 23);
+      ref = new_ref;
       if (__any_sync(0xffffffffu, need)) {
         if (ok) ok = mbar_wait(bar(C::kBarPVDone), (it - 1) & 1, abort_flag);
         tc_fence_after();
-        const float a = upd ? alpha : 1.0f;
         uint32_t r[32];
 #pragma unroll
         for (int ch = 0; ch < 2; ++ch) {
@@ -305,13 +313,12 @@ __global__ void __launch_bounds__(320, 1) attn_qbsa_kernel(const __grid_constant
         if (half == 0) tmem_st1(l_col, __float_as_uint(__uint_as_float(tmem_ld1_wait(l_col)) * a));
         tmem_st_wait();
       }
-      m = m_new;
       uint32_t pk[16];
 #pragma unroll
       for (int x = 0; x < 16; ++x) {
         float pv[4];
 #pragma unroll
-        for (int y = 0; y < 4; ++y) pv[y] = ex2(fmaf(sv[4 * x + y], cst, -m));
+        for (int y = 0; y < 4; ++y) pv[y] = ex2(fmaf(sv[4 * x + y], cst, -ref));
         pk[x] = pack_e4m3x4(pv[0], pv[1], pv[2], pv[3]);
       }
       tmem_st16(tmem + lane_off + (bi ? C::kColP1 : C::kColP0) + half * 16, pk);
@@ -362,7 +369,7 @@ __global__ void __launch_bounds__(320, 1) attn_qbsa_kernel(const __grid_constant
       const int64_t sidx = ((int64_t)b * p.Nq + h) * p.Sq + i_glob;
       const bool live = l > 0.f;
       if (p.softmax_max) p.softmax_max[sidx] = live ? m * 0.6931471805599453f : kNegInf;
-      if (p.softmax_sum) p.softmax_sum[sidx] = live ? l : 0.f;
+      if (p.softmax_sum) p.softmax_sum[sidx] = live ? l * ex2(ref - m) : 0.f;  // against the true max
     }
   }
 
