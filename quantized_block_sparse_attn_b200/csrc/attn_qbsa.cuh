@@ -64,7 +64,7 @@ struct QbsaCfg {
   static constexpr int kOnesOff = kVOff + kStages * kTileBytes;  // 16 x 128 bytes of E4M3 1.0
   static constexpr int kCOff = kOnesOff + 2048;                   // float dequant constant per kept block
   static constexpr int kListOff = kCOff + kQbsaMaxKBlocks * 4;    // uint16 kept-block list
-  static constexpr int kXOff = kListOff + kQbsaMaxKBlocks * 2;    // int row-max exchange [2][2][128]
+  static constexpr int kXOff = kListOff + kQbsaMaxKBlocks * 2;    // float running max / reference [2][2][128]
   static constexpr int kBarOff = kXOff + 2 * 2 * 128 * 4;
   static constexpr int kBarQFull = 0;
   static constexpr int kBarKFull = 1;
@@ -76,7 +76,8 @@ struct QbsaCfg {
   static constexpr int kBarPFull = kBarSFree + 2;
   static constexpr int kBarPVDone = kBarPFull + 2;
   static constexpr int kBarOFinal = kBarPVDone + 1;  // last P·V done (single use)
-  static constexpr int kNumBars = kBarOFinal + 1;
+  static constexpr int kBarMH = kBarOFinal + 1;      // [parity][quarter] running-max hand-over
+  static constexpr int kNumBars = kBarMH + 8;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // tmem addr, abort flag, list count
   static constexpr int kSmemBytes = kMiscOff + 16 + 1024;
   static constexpr uint32_t kTmemCols = 512;
@@ -152,11 +153,12 @@ __global__ void __launch_bounds__(320, 1) attn_qbsa_kernel(const __grid_constant
       }
       for (int b2 = 0; b2 < 2; ++b2) {
         mbar_init(bar(C::kBarSFull + b2), 1);
-        mbar_init(bar(C::kBarSFree + b2), C::kSoftmaxThreads);
-        mbar_init(bar(C::kBarPFull + b2), C::kSoftmaxThreads);
+        mbar_init(bar(C::kBarSFree + b2), C::kSoftmaxThreads / 2);  // the 4 warps of that parity
+        mbar_init(bar(C::kBarPFull + b2), C::kSoftmaxThreads / 2);
       }
       mbar_init(bar(C::kBarPVDone), 1);
       mbar_init(bar(C::kBarOFinal), 1);
+      for (int i = 0; i < 8; ++i) mbar_init(bar(C::kBarMH + i), 32);
       fence_mbar_init();
       tma_prefetch_desc(&p.tm_q);
       tma_prefetch_desc(&p.tm_k);
@@ -246,88 +248,119 @@ __global__ void __launch_bounds__(320, 1) attn_qbsa_kernel(const __grid_constant
     }
   } else {
     // ---------------------------------------------------------------- softmax warps
+    // The two warps of a TMEM lane quarter (the same 32 query rows) take alternate
+    // steps of the kept-block list, each with all 128 key columns: parity 0 the even
+    // steps (S0 / P0), parity 1 the odd steps (S1 / P1).  Per step they hand the running
+    // max and the reference to each other through shared memory and a per-quarter
+    // mbarrier, so one warp's load / max phase overlaps the other's ex2 phase.
     const int quarter = warp & 3;
-    const int half = (warp - 2) >> 2;  // 0: key columns [0,64), 1: [64,128)
+    const int par = (warp - 2) >> 2;
     const int row = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const int64_t i_glob = (int64_t)qb * kTile + row;
     const float kNegInf = -__int_as_float(0x7f800000);
-    const uint32_t o_col = tmem + lane_off + C::kColO + half * 64;
+    const uint32_t o_col = tmem + lane_off + C::kColO;
     const uint32_t l_col = tmem + lane_off + C::kColL;
+    const uint32_t s_col = tmem + lane_off + (par ? C::kColS1 : C::kColS0);
+    const uint32_t p_col = tmem + lane_off + (par ? C::kColP1 : C::kColP0);
+    const uint32_t mh_mine = bar(C::kBarMH + par * 4 + quarter);
+    const uint32_t mh_other = bar(C::kBarMH + (par ^ 1) * 4 + quarter);
+    float* m_pub = xch;        // [parity][row] running max after that warp's latest step
+    float* r_pub = xch + 256;  // [parity][row] reference after that step
 
     float m = kNegInf;    // running max, log2 domain
     float ref = kNegInf;  // power-of-two reference of the FP8 weights (an integer)
     bool ok = true;
-    for (int it = 0; it < n; ++it) {
+    for (int it = par; it < n; it += 2) {
       const int kb = list[it];
-      const int bi = it & 1;
       const float cst = cst_list[it];
-      const int valid = min(kTile, p.Skv - kb * kTile) - half * 64;  // valid columns of this half
-      // never leave the loop early (the paired warp waits on named barriers below)
-      if (ok) ok = mbar_wait(bar(C::kBarSFull + bi), (it >> 1) & 1, abort_flag);
+      const int valid = min(kTile, p.Skv - kb * kTile);
+      if (ok) ok = mbar_wait(bar(C::kBarSFull + par), (it >> 1) & 1, abort_flag);
       tc_fence_after();
-      float sv[64];  // exact: |dot| <= 128 * 127^2 < 2^24
-      {
-        uint32_t r[64];
-        tmem_ld64_wait(tmem + lane_off + (bi ? C::kColS1 : C::kColS0) + half * 64, r);
-#pragma unroll
-        for (int x = 0; x < 64; ++x) sv[x] = __int2float_rn(static_cast<int32_t>(r[x]));
-      }
+      uint32_t r[128];  // s32 dot products, |t| <= 128 * 127^2 < 2^24 (exact in f32)
+      tmem_ld128_wait(s_col, r);
       tc_fence_before();
-      mbar_arrive(bar(C::kBarSFree + bi));
-
-      if (valid < 64) {  // tail block: keys past S_kv get -inf (p = 0 below)
+      mbar_arrive(bar(C::kBarSFree + par));
+      if (valid < kTile) {  // tail block: keys past S_kv
 #pragma unroll
-        for (int x = 0; x < 64; ++x)
-          if (x >= valid) sv[x] = kNegInf;
+        for (int x = 0; x < 128; ++x)
+          if (x >= valid) r[x] = 0x80000000u;
       }
-      const float pmax = max64(sv);
-      float* slot = xch + (it & 1) * 256;
-      slot[half * 128 + row] = pmax;
-      qbsa_named_bar_sync(1 + quarter, 64);
-      const float tmax = fmaxf(pmax, slot[(half ^ 1) * 128 + row]);
-
+      int32_t acc[8];  // eight independent max chains, then a 3-level tree
+#pragma unroll
+      for (int x = 0; x < 8; ++x) acc[x] = static_cast<int32_t>(r[x]);
+#pragma unroll
+      for (int x = 8; x < 128; ++x) acc[x & 7] = max(acc[x & 7], static_cast<int32_t>(r[x]));
+      const int32_t tmax = max(max(max(acc[0], acc[1]), max(acc[2], acc[3])), max(max(acc[4], acc[5]), max(acc[6], acc[7])));
       // max(t) * c == max(t * c): multiplication by c > 0 is monotone in float
-      const float m_blk = tmax * cst;
-      m = fmaxf(m, m_blk);
+      const float m_blk = __int2float_rn(tmax) * cst;
+      float m_prev = kNegInf, ref_prev = kNegInf;
+      if (it > 0) {
+        if (ok) ok = mbar_wait(mh_other, ((it - 1) >> 1) & 1, abort_flag);
+        m_prev = m_pub[(par ^ 1) * 128 + row];
+        ref_prev = r_pub[(par ^ 1) * 128 + row];
+      }
+      m = fmaxf(m_prev, m_blk);
       // power-of-two reference: re-set to ceil(m) once m exceeds it by more than 8, so
       // p <= 2^8 stays below E4M3's 448 and every rescale is an exact power of two
-      const bool upd = (ref == kNegInf) || (m > ref + 8.0f);
-      const float new_ref = upd ? ceilf(m) : ref;
-      const bool need = upd && (ref != kNegInf);
-      // 2^(ref - new_ref) built from its exponent bits (exact; flush below 2^-126)
-      const int dexp = need ? static_cast<int>(ref - new_ref) : 0;
-      const float a = (dexp < -126) ? 0.f : __int_as_float((127 + dexp) << 23);
-      ref = new_ref;
+      const bool upd = (ref_prev == kNegInf) || (m > ref_prev + 8.0f);
+      ref = upd ? ceilf(m) : ref_prev;
+      m_pub[par * 128 + row] = m;
+      r_pub[par * 128 + row] = ref;
+      mbar_arrive(mh_mine);  // release: the values above are visible to the other warp
+      const bool need = upd && (ref_prev != kNegInf);
       if (__any_sync(0xffffffffu, need)) {
+        // 2^(ref_prev - ref) built from its exponent bits (exact; flush below 2^-126)
+        const int dexp = need ? static_cast<int>(ref_prev - ref) : 0;
+        const float a = (dexp < -126) ? 0.f : __int_as_float((127 + dexp) << 23);
         if (ok) ok = mbar_wait(bar(C::kBarPVDone), (it - 1) & 1, abort_flag);
         tc_fence_after();
-        uint32_t r[32];
+        uint32_t o[32];
+#pragma unroll 1
+        for (int ch = 0; ch < 4; ++ch) {
+          tmem_ld32_wait(o_col + ch * 32, o);
 #pragma unroll
-        for (int ch = 0; ch < 2; ++ch) {
-          tmem_ld32_wait(o_col + ch * 32, r);
-#pragma unroll
-          for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(__uint_as_float(r[x]) * a);
-          tmem_st32(o_col + ch * 32, r);
+          for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * a);
+          tmem_st32(o_col + ch * 32, o);
+          tmem_st_wait();
         }
-        if (half == 0) tmem_st1(l_col, __float_as_uint(__uint_as_float(tmem_ld1_wait(l_col)) * a));
+        tmem_st1(l_col, __float_as_uint(__uint_as_float(tmem_ld1_wait(l_col)) * a));
         tmem_st_wait();
       }
-      uint32_t pk[16];
+      // weights p = 2^(t c - ref) -> E4M3, eight packed columns per TMEM store
 #pragma unroll
-      for (int x = 0; x < 16; ++x) {
-        float pv[4];
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t pk[8];
 #pragma unroll
-        for (int y = 0; y < 4; ++y) pv[y] = ex2(fmaf(sv[4 * x + y], cst, -ref));
-        pk[x] = pack_e4m3x4(pv[0], pv[1], pv[2], pv[3]);
+        for (int x = 0; x < 8; ++x) {
+          const int e = ch * 32 + 4 * x;
+          pk[x] = pack_e4m3x4(ex2(fmaf(__int2float_rn(static_cast<int32_t>(r[e])), cst, -ref)),
+                              ex2(fmaf(__int2float_rn(static_cast<int32_t>(r[e + 1])), cst, -ref)),
+                              ex2(fmaf(__int2float_rn(static_cast<int32_t>(r[e + 2])), cst, -ref)),
+                              ex2(fmaf(__int2float_rn(static_cast<int32_t>(r[e + 3])), cst, -ref)));
+          if (valid < kTile) {  // keys past S_kv weigh exactly 0
+            uint32_t keep = 0;
+#pragma unroll
+            for (int y = 0; y < 4; ++y)
+              if (e + y < valid) keep |= 0xFFu << (8 * y);
+            pk[x] &= keep;
+          }
+        }
+        tmem_st8(p_col + ch * 8, pk);
       }
-      tmem_st16(tmem + lane_off + (bi ? C::kColP1 : C::kColP0) + half * 16, pk);
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(bar(C::kBarPFull + bi));
+      mbar_arrive(bar(C::kBarPFull + par));
+    }
+    // the final running max and reference come from the warp that ran the last step
+    if (n > 0 && ((n - 1) & 1) != par) {
+      if (ok) ok = mbar_wait(mh_other, ((n - 1) >> 1) & 1, abort_flag);
+      m = m_pub[(par ^ 1) * 128 + row];
+      ref = r_pub[(par ^ 1) * 128 + row];
     }
 
-    // ------------------------------------------------------------ epilogue
+    // ------------------------------------------------------------ epilogue (O columns 64*par..)
+    const int half = par;
     const bool row_valid = i_glob < p.Sq;
     bool have_o = ok && n > 0;
     if (have_o) {
@@ -344,7 +377,7 @@ __global__ void __launch_bounds__(320, 1) attn_qbsa_kernel(const __grid_constant
     for (int ch = 0; ch < 2; ++ch) {
       uint32_t r[32];
       if (have_o) {
-        tmem_ld32_wait(o_col + ch * 32, r);
+        tmem_ld32_wait(o_col + half * 64 + ch * 32, r);
       } else {
 #pragma unroll
         for (int x = 0; x < 32; ++x) r[x] = 0u;
