@@ -291,13 +291,8 @@ __global__ void __launch_bounds__(320, 1) attn_qbsa_kernel(const __grid_constant
 
     // columns of step i that lie inside S_kv, in this half
     auto valid_cols = [&](int i) -> int { return min(kTile, p.Skv - static_cast<int>(list[i]) * kTile) - half * 64; };
-    // load this half of S(i) (raw s32), release the buffer, mask the tail
-    auto load_s = [&](int i, uint32_t (&r)[64], bool& ok) {
-      if (ok) ok = mbar_wait(bar(C::kBarSFull + (i & 1)), (i >> 1) & 1, abort_flag);
-      tc_fence_after();
-      tmem_ld64_wait(tmem + lane_off + ((i & 1) ? C::kColS1 : C::kColS0) + half * 64, r);
-      tc_fence_before();
-      mbar_arrive(bar(C::kBarSFree + (i & 1)));
+    auto s_addr = [&](int i) -> uint32_t { return tmem + lane_off + ((i & 1) ? C::kColS1 : C::kColS0) + half * 64; };
+    auto mask_tail = [&](int i, uint32_t (&r)[64]) {
       const int valid = valid_cols(i);
       if (valid < 64) {
 #pragma unroll
@@ -305,19 +300,17 @@ __global__ void __launch_bounds__(320, 1) attn_qbsa_kernel(const __grid_constant
           if (x >= valid) r[x] = 0x80000000u;  // INT32_MIN: below every real dot product
       }
     };
-    // row max of step i from this half's partial max (exchange with the paired warp)
-    auto row_max = [&](int i, int32_t pmax) -> int32_t {
-      int32_t* slot = xch + (i & 1) * 256;
-      slot[half * 128 + row] = pmax;
+    // the paired warp's partial row max of step i (both halves published theirs first)
+    auto publish_max = [&](int i, int32_t pmax) { xch[(i & 1) * 256 + half * 128 + row] = pmax; };
+    auto combine_max = [&](int i, int32_t pmax) -> int32_t {
       qbsa_named_bar_sync(1 + quarter, 64);
-      return max(pmax, slot[(half ^ 1) * 128 + row]);
+      return max(pmax, xch[(i & 1) * 256 + (half ^ 1) * 128 + row]);
     };
 
     float m = kNegInf;    // running max, log2 domain
     float ref = kNegInf;  // power-of-two reference of the FP8 weights (an integer)
     float resc = 1.0f;    // pending exact O / L rescale for the current step
     bool ok = true;
-    uint32_t rc[64];      // raw S of the current step
     // decide the reference for step i from its row max; sets the pending rescale
     auto step_ref = [&](int i, int32_t tmax) {
       // max(t) * c == max(t * c): multiplication by c > 0 is monotone in float
@@ -333,44 +326,66 @@ __global__ void __launch_bounds__(320, 1) attn_qbsa_kernel(const __grid_constant
       }
       ref = new_ref;
     };
+    uint32_t ra[64], rb[64];  // raw S of the current and the next step
     if (n > 0) {
-      load_s(0, rc, ok);
-      step_ref(0, row_max(0, imax64(rc)));
+      if (ok) ok = mbar_wait(bar(C::kBarSFull), 0, abort_flag);
+      tc_fence_after();
+      tmem_ld64_issue(s_addr(0), ra);
+      tmem_ld64_wait(ra);
+      tc_fence_before();
+      mbar_arrive(bar(C::kBarSFree));
+      mask_tail(0, ra);
+      const int32_t pm = imax64(ra);
+      publish_max(0, pm);
+      step_ref(0, combine_max(0, pm));
     }
-    // never leave the loop early: the paired warp waits on the named barrier of row_max
-    for (int it = 0; it < n; ++it) {
+    // One step: weights of step it from rc, while S(it+1) streams into rn.  Never leaves
+    // early: the paired warp waits on the named barrier in combine_max.
+    // E4M3 weights of the 32 columns [c0, c0+32) of step it, stored to its P buffer
+    auto weights32 = [&](int it, const uint32_t (&rc)[64], int c0, float cst, int valid) {
+      uint32_t pk[8];
+#pragma unroll
+      for (int x = 0; x < 8; ++x) {
+        const int e = c0 + 4 * x;
+        pk[x] = pack_e4m3x4(ex2(fmaf(__int2float_rn(static_cast<int32_t>(rc[e])), cst, -ref)),
+                            ex2(fmaf(__int2float_rn(static_cast<int32_t>(rc[e + 1])), cst, -ref)),
+                            ex2(fmaf(__int2float_rn(static_cast<int32_t>(rc[e + 2])), cst, -ref)),
+                            ex2(fmaf(__int2float_rn(static_cast<int32_t>(rc[e + 3])), cst, -ref)));
+        if (valid < 64) {  // keys past S_kv weigh exactly 0
+          uint32_t keep = 0;
+#pragma unroll
+          for (int y = 0; y < 4; ++y)
+            if (e + y < valid) keep |= 0xFFu << (8 * y);
+          pk[x] &= keep;
+        }
+      }
+      tmem_st8(tmem + lane_off + ((it & 1) ? C::kColP1 : C::kColP0) + half * 16 + c0 / 4, pk);
+    };
+    auto step = [&](int it, uint32_t (&rc)[64], uint32_t (&rn)[64]) {
       const bool has_next = it + 1 < n;
-      uint32_t rn[64];
+      // P buffer it & 1 was read by P·V(it-2)
+      if (it >= 2 && ok) ok = mbar_wait(bar(C::kBarPFree + (it & 1)), ((it - 2) >> 1) & 1, abort_flag);
+      tc_fence_after();
+      const float cst = cst_list[it];
+      const int valid = valid_cols(it);
+      weights32(it, rc, 0, cst, valid);
       if (has_next) {
-        load_s(it + 1, rn, ok);
+        if (ok) ok = mbar_wait(bar(C::kBarSFull + ((it + 1) & 1)), ((it + 1) >> 1) & 1, abort_flag);
+        tc_fence_after();
+        tmem_ld64_issue(s_addr(it + 1), rn);  // completes while the second half is computed
+      }
+      weights32(it, rc, 32, cst, valid);
+      if (has_next) {
+        tmem_ld64_wait(rn);
+        tc_fence_before();
+        mbar_arrive(bar(C::kBarSFree + ((it + 1) & 1)));
+        mask_tail(it + 1, rn);
       } else {
 #pragma unroll
         for (int x = 0; x < 64; ++x) rn[x] = 0x80000000u;
       }
-      // weights of step it (ex2) interleaved with the row max of step it+1 (integer)
-      const float cst = cst_list[it];
-      uint32_t pk[16];
-#pragma unroll
-      for (int x = 0; x < 16; ++x) {
-        pk[x] = pack_e4m3x4(ex2(fmaf(__int2float_rn(static_cast<int32_t>(rc[4 * x])), cst, -ref)),
-                            ex2(fmaf(__int2float_rn(static_cast<int32_t>(rc[4 * x + 1])), cst, -ref)),
-                            ex2(fmaf(__int2float_rn(static_cast<int32_t>(rc[4 * x + 2])), cst, -ref)),
-                            ex2(fmaf(__int2float_rn(static_cast<int32_t>(rc[4 * x + 3])), cst, -ref)));
-      }
       const int32_t pmax_next = imax64(rn);
-      const int valid = valid_cols(it);
-      if (valid < 64) {  // keys past S_kv weigh exactly 0
-#pragma unroll
-        for (int x = 0; x < 16; ++x) {
-          uint32_t keep = 0;
-#pragma unroll
-          for (int y = 0; y < 4; ++y)
-            if (4 * x + y < valid) keep |= 0xFFu << (8 * y);
-          pk[x] &= keep;
-        }
-      }
-      // P buffer it & 1 was read by P·V(it-2)
-      if (it >= 2 && ok) ok = mbar_wait(bar(C::kBarPFree + (it & 1)), ((it - 2) >> 1) & 1, abort_flag);
+      if (has_next) publish_max(it + 1, pmax_next);
       // pending rescale of O and L (reference moved at this step): after P·V(it-1)
       if (__any_sync(0xffffffffu, resc != 1.0f)) {
         if (ok) ok = mbar_wait(bar(C::kBarPVDone), (it - 1) & 1, abort_flag);
@@ -387,14 +402,17 @@ __global__ void __launch_bounds__(320, 1) attn_qbsa_kernel(const __grid_constant
         if (half == 0) tmem_st1(l_col, __float_as_uint(__uint_as_float(tmem_ld1_wait(l_col)) * resc));
         tmem_st_wait();
       }
-      tc_fence_after();
-      tmem_st16(tmem + lane_off + ((it & 1) ? C::kColP1 : C::kColP0) + half * 16, pk);
-      tmem_st_wait();
+      tmem_st_wait();  // both halves of P(it) are in TMEM
       tc_fence_before();
       mbar_arrive(bar(C::kBarPFull + (it & 1)));
-      if (has_next) step_ref(it + 1, row_max(it + 1, pmax_next));
+      if (has_next) step_ref(it + 1, combine_max(it + 1, pmax_next));
+    };
+    // (a register copy per step: unrolling by two to alternate the arrays spills registers,
+    // and the asynchronously loaded array must never be spilled before its wait)
+    for (int it = 0; it < n; ++it) {
+      step(it, ra, rb);
 #pragma unroll
-      for (int x = 0; x < 64; ++x) rc[x] = rn[x];
+      for (int x = 0; x < 64; ++x) ra[x] = rb[x];
     }
 
     // ------------------------------------------------------------ epilogue

@@ -242,6 +242,31 @@ __device__ __forceinline__ void tmem_ld64_wait(uint32_t taddr, uint32_t (&r)[64]
       : "memory");
 }
 
+// Issue a load of 64 consecutive 32-bit columns without waiting.  The registers are
+// undefined until tmem_ld64_wait(r) on the same array; that wait takes them as
+// read-write operands, so no use of them can be scheduled before it.
+__device__ __forceinline__ void tmem_ld64_issue(uint32_t taddr, uint32_t (&r)[64]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,"
+      "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+      "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];"
+      : QBSA_R8(0), QBSA_R8(8), QBSA_R8(16), QBSA_R8(24), QBSA_R8(32), QBSA_R8(40), QBSA_R8(48), QBSA_R8(56)
+      : "r"(taddr)
+      : "memory");
+}
+#define QBSA_RW8(i) "+r"(r[i]), "+r"(r[i + 1]), "+r"(r[i + 2]), "+r"(r[i + 3]), "+r"(r[i + 4]), "+r"(r[i + 5]), \
+                    "+r"(r[i + 6]), "+r"(r[i + 7])
+__device__ __forceinline__ void tmem_ld64_wait(uint32_t (&r)[64]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : QBSA_RW8(0), QBSA_RW8(8), QBSA_RW8(16), QBSA_RW8(24), QBSA_RW8(32), QBSA_RW8(40), QBSA_RW8(48),
+                 QBSA_RW8(56)
+               :
+               : "memory");
+}
+#undef QBSA_RW8
+
 // Load 128 consecutive 32-bit columns (two 64-column loads, one wait).
 __device__ __forceinline__ void tmem_ld128_wait(uint32_t taddr, uint32_t (&r)[128]) {
   asm volatile(
