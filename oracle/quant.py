@@ -35,8 +35,10 @@ Readings where the article is silent (each also listed in the design notes):
   reference makes the rescaling exact, and E4M3 rounding commutes with powers of two,
   so the codes equal those against the final max except for weights in E4M3's
   subnormal range (below 2^-6 of the reference).
-* p is held in float32 (the precision in which the FP8 decision is taken) and
-  rounded to E4M3 (nearest even): p8 = E4M3(p).  l = Σ p8 (the sum of the ROUNDED
+* p is held in FP16 before its FP8 rounding, the precision the article gives for P
+  (section "昇腾亲和的量化叠加稀疏Attention算子优化": the FP16 P matrix is converted
+  to FP8): p16 = FP16(2^(z - R)) and p8 = E4M3(p16), both nearest even; the FP8
+  decision is taken on p16 on both sides.  l = Σ p8 (the sum of the ROUNDED
   weights, so constant V returns V exactly); O[:, c] = acc[:, c] / l · v_scale[c]
   with acc = Σ p8 · v8.
 * softmax_max = final m in the natural-log domain (max s) and softmax_sum = l · 2^(R - m):
@@ -132,7 +134,7 @@ def _head_forward(q8, k8, qs, ks, v8f, vs, mask_rows, scale, qbs, round_p=True):
             l, acc, ref = l * alpha, acc * alpha[:, None], new_ref
             p = np.exp2(z - ref[:, None])
             if round_p:
-                p = e4m3_decode(e4m3_encode(p.astype(np.float32)))
+                p = e4m3_decode(e4m3_encode(p.astype(np.float16).astype(np.float32)))
             l = l + p.sum(axis=1)
             acc = acc + p @ v8f[c0:c1]
         live = l > 0
@@ -214,7 +216,8 @@ def qbsa_forward_loops(q8, k8, q_scale, k_scale, v8, v_scale, block_mask, scale:
                         acc = [a * alpha for a in acc]
                         ref = new_ref
                     for j, zj in zip(cols, z):
-                        p = float(e4m3_decode(e4m3_encode(np.float32(2.0 ** (zj - ref)))))
+                        p16 = np.float16(2.0 ** (zj - ref))           # P held in FP16 first
+                        p = float(e4m3_decode(e4m3_encode(np.float32(p16))))
                         l += p
                         vrow = e4m3_decode(v8[b, g, j])
                         for c in range(D):

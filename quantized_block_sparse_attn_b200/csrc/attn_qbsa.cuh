@@ -10,19 +10,17 @@
 // One CTA per (batch, head, 128-row query block).  Warp 0 first compacts the CTA's row
 // of the block mask into the ascending list of kept key blocks in shared memory, with
 // each block's dequantisation constant s_q * s_k * scale * log2(e).  Then:
-//   warp 0      TMA producer: Q once; K of step j+2 ahead of V of step j (3-stage rings).
-//   warp 1      TMEM owner + MMA issuer, S two steps ahead of P·V:
-//               S(j+2) = Q8 K8ᵀ (kind::i8, s32 in TMEM) as soon as S(j) has been read,
-//               then O += P8(j) V8 (kind::f8f6f4, A = P8 from TMEM, B = V8 MN-major) and
-//               L += P8(j) · 1 (N = 16 ones matrix), so L is exactly Σ p8.
-//   warps 2..9  softmax, two warps per TMEM lane quarter (the same 32 query rows), each
-//               owning 64 of the 128 key columns.  Software-pipelined by one step: in
-//               step it a thread loads S(it+1) and computes its row max while it turns
-//               S(it) into weights, so integer and ex2 work overlap.  Weights
-//               p = 2^(t c - R) use a power-of-two reference R re-set to ceil(running
-//               max) only when the max exceeds it by more than 8; the O / L rescale
-//               that goes with it (an exact power of two, rare) runs just before P is
-//               published, when the previous P·V has long finished.
+//   warp 0      TMA producer (Q once; K and V tiles of kept blocks, 3-stage rings)
+//   warp 1      TMEM owner + MMA issuer: S = Q8 K8ᵀ (kind::i8, s32 in TMEM);
+//               O += P8 V8 (kind::f8f6f4, A = P8 from TMEM, B = V8 MN-major) and
+//               L += P8 · 1 (N = 16 ones matrix), so L is exactly Σ p8.
+//   warps 2..9  softmax: query row 32*(warp%4)+lane; warps 2..5 own key columns [0,64),
+//               warps 6..9 [64,128), exchanging partial row maxima through shared
+//               memory.  Exact s32 -> f32 (|dot| < 2^24), online softmax whose weights
+//               p = 2^(z - R) use a power-of-two reference R re-set to ceil(running max)
+//               only when the max exceeds it by more than 8 (exact power-of-two
+//               rescales of O and L, rare), P -> E4M3 into TMEM, epilogue
+//               O * v_scale / L -> bf16.
 // TMEM columns: S0 [0,128) S1 [128,256) O [256,384) L [384,400) P0 [448,480) P1 [480,512).
 //
 // CTA order: query heads in groups whose K8/V8 fit in about 48 MB of L2, query blocks
@@ -73,12 +71,11 @@ struct QbsaCfg {
   static constexpr int kBarKEmpty = kBarKFull + kStages;
   static constexpr int kBarVFull = kBarKEmpty + kStages;
   static constexpr int kBarVEmpty = kBarVFull + kStages;
-  static constexpr int kBarSFull = kBarVEmpty + kStages;  // [2]
-  static constexpr int kBarSFree = kBarSFull + 2;         // [2]
-  static constexpr int kBarPFull = kBarSFree + 2;         // [2]
-  static constexpr int kBarPFree = kBarPFull + 2;         // [2]: P·V that read P buffer b finished
-  static constexpr int kBarPVDone = kBarPFree + 2;        // every P·V
-  static constexpr int kBarOFinal = kBarPVDone + 1;       // last P·V done (single use)
+  static constexpr int kBarSFull = kBarVEmpty + kStages;
+  static constexpr int kBarSFree = kBarSFull + 2;
+  static constexpr int kBarPFull = kBarSFree + 2;
+  static constexpr int kBarPVDone = kBarPFull + 2;
+  static constexpr int kBarOFinal = kBarPVDone + 1;  // last P·V done (single use)
   static constexpr int kNumBars = kBarOFinal + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // tmem addr, abort flag, list count
   static constexpr int kSmemBytes = kMiscOff + 16 + 1024;
@@ -106,16 +103,6 @@ __device__ __forceinline__ void qbsa_named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
-// Largest of 64 int32 values: eight independent chains, then a 3-level tree.
-__device__ __forceinline__ int32_t imax64(const uint32_t (&r)[64]) {
-  int32_t a[8];
-#pragma unroll
-  for (int x = 0; x < 8; ++x) a[x] = static_cast<int32_t>(r[x]);
-#pragma unroll
-  for (int x = 8; x < 64; ++x) a[x & 7] = max(a[x & 7], static_cast<int32_t>(r[x]));
-  return max(max(max(a[0], a[1]), max(a[2], a[3])), max(max(a[4], a[5]), max(a[6], a[7])));
-}
-
 __global__ void __launch_bounds__(320, 1) attn_qbsa_kernel(const __grid_constant__ QbsaParams p) {
   using C = QbsaCfg;
   extern __shared__ uint8_t smem_raw[];
@@ -132,7 +119,7 @@ __global__ void __launch_bounds__(320, 1) attn_qbsa_kernel(const __grid_constant
   int* count_slot = reinterpret_cast<int*>(smem + C::kMiscOff + 8);
   uint16_t* list = reinterpret_cast<uint16_t*>(smem + C::kListOff);
   float* cst_list = reinterpret_cast<float*>(smem + C::kCOff);
-  int32_t* xch = reinterpret_cast<int32_t*>(smem + C::kXOff);
+  float* xch = reinterpret_cast<float*>(smem + C::kXOff);
 
   // head groups (L2 reuse of K/V), query blocks in order, heads fastest inside a group
   const int64_t per_group = (int64_t)p.head_grp * p.n_rank;
@@ -140,10 +127,10 @@ __global__ void __launch_bounds__(320, 1) attn_qbsa_kernel(const __grid_constant
   const int h0 = grp * p.head_grp;
   const int hcount = min(p.head_grp, p.Nq - h0);
   const int off = static_cast<int>(blockIdx.x - grp * per_group);
-  const int r_idx = off / hcount;
+  const int r = off / hcount;
   const int h = h0 + off % hcount;
-  const int qb = r_idx % p.nqb;
-  const int b = r_idx / p.nqb;
+  const int qb = r % p.nqb;
+  const int b = r / p.nqb;
   const int g = h / p.group;
 
   if (warp == 0) {
@@ -167,7 +154,6 @@ __global__ void __launch_bounds__(320, 1) attn_qbsa_kernel(const __grid_constant
         mbar_init(bar(C::kBarSFull + b2), 1);
         mbar_init(bar(C::kBarSFree + b2), C::kSoftmaxThreads);
         mbar_init(bar(C::kBarPFull + b2), C::kSoftmaxThreads);
-        mbar_init(bar(C::kBarPFree + b2), 1);
       }
       mbar_init(bar(C::kBarPVDone), 1);
       mbar_init(bar(C::kBarOFinal), 1);
@@ -193,34 +179,21 @@ __global__ void __launch_bounds__(320, 1) attn_qbsa_kernel(const __grid_constant
 
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
-    // consumption order is S(0) S(1) S(2) PV(0) S(3) PV(1) ...: K runs two steps ahead of V
     if (lane == 0 && n > 0) {
       const uint64_t pol_q = l2_policy_evict_first();
       const uint64_t pol_kv = l2_policy_evict_last();
       mbar_arrive_expect_tx(bar(C::kBarQFull), C::kTileBytes);
       tma_load_4d(base + C::kQOff, &p.tm_q, bar(C::kBarQFull), 0, qb * kTile, h, b, pol_q);
-      auto load_k = [&](int i) -> bool {
-        const int s = i % C::kStages;
-        if (i >= C::kStages && !mbar_wait(bar(C::kBarKEmpty + s), ((i / C::kStages) & 1) ^ 1, abort_flag))
-          return false;
+      for (int it = 0; it < n; ++it) {
+        const int s = it % C::kStages;
+        const uint32_t ph = (it / C::kStages) & 1;
+        const int kv_row = static_cast<int>(list[it]) * kTile;
+        if (it >= C::kStages && !mbar_wait(bar(C::kBarKEmpty + s), ph ^ 1, abort_flag)) break;
         mbar_arrive_expect_tx(bar(C::kBarKFull + s), C::kTileBytes);
-        tma_load_4d(base + C::kKOff + s * C::kTileBytes, &p.tm_k, bar(C::kBarKFull + s), 0,
-                    static_cast<int>(list[i]) * kTile, g, b, pol_kv);
-        return true;
-      };
-      auto load_v = [&](int i) -> bool {
-        const int s = i % C::kStages;
-        if (i >= C::kStages && !mbar_wait(bar(C::kBarVEmpty + s), ((i / C::kStages) & 1) ^ 1, abort_flag))
-          return false;
+        tma_load_4d(base + C::kKOff + s * C::kTileBytes, &p.tm_k, bar(C::kBarKFull + s), 0, kv_row, g, b, pol_kv);
+        if (it >= C::kStages && !mbar_wait(bar(C::kBarVEmpty + s), ph ^ 1, abort_flag)) break;
         mbar_arrive_expect_tx(bar(C::kBarVFull + s), C::kTileBytes);
-        tma_load_4d(base + C::kVOff + s * C::kTileBytes, &p.tm_v, bar(C::kBarVFull + s), 0,
-                    static_cast<int>(list[i]) * kTile, g, b, pol_kv);
-        return true;
-      };
-      bool ok = load_k(0) && (n < 2 || load_k(1));
-      for (int j = 0; ok && j < n; ++j) {
-        if (j + 2 < n && !load_k(j + 2)) break;
-        if (!load_v(j)) break;
+        tma_load_4d(base + C::kVOff + s * C::kTileBytes, &p.tm_v, bar(C::kBarVFull + s), 0, kv_row, g, b, pol_kv);
       }
     }
   } else if (warp == 1) {
@@ -230,37 +203,12 @@ __global__ void __launch_bounds__(320, 1) attn_qbsa_kernel(const __grid_constant
       constexpr uint32_t idesc_pv = idesc_e4m3(128, 128, true);
       constexpr uint32_t idesc_pl = idesc_e4m3(128, 16, false);
       const uint32_t ones = base + C::kOnesOff;
-      const uint32_t qbase = base + C::kQOff;
-      auto issue_s = [&](int i) -> bool {  // S(i) into buffer i & 1
-        const int s = i % C::kStages;
-        const int bi = i & 1;
-        if (!mbar_wait(bar(C::kBarKFull + s), (i / C::kStages) & 1, abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t kbase = base + C::kKOff + s * C::kTileBytes;
-        const uint32_t scol = bi ? C::kColS1 : C::kColS0;
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          mma_i8_ss(tmem + scol, sdesc_sw128(qbase + kk * 32, 16, 1024), sdesc_sw128(kbase + kk * 32, 16, 1024),
-                    idesc_qk, kk > 0 ? 1u : 0u);
-        }
-        mma_commit(bar(C::kBarSFull + bi));
-        mma_commit(bar(C::kBarKEmpty + s));
-        return true;
-      };
       bool ok = mbar_wait(bar(C::kBarQFull), 0, abort_flag);
-      if (ok) ok = issue_s(0);
-      if (ok && n > 1) ok = issue_s(1);
-      for (int j = 0; ok && j < n; ++j) {
+      auto issue_pv = [&](int j) -> bool {
         const int bj = j & 1;
-        // S(j+2) reuses buffer j & 1 once the softmax warps have read S(j)
-        if (j + 2 < n) {
-          if (!mbar_wait(bar(C::kBarSFree + bj), (j >> 1) & 1, abort_flag)) { ok = false; break; }
-          if (!issue_s(j + 2)) { ok = false; break; }
-        }
-        // P·V of step j
         const int s = j % C::kStages;
-        if (!mbar_wait(bar(C::kBarPFull + bj), (j >> 1) & 1, abort_flag)) { ok = false; break; }
-        if (!mbar_wait(bar(C::kBarVFull + s), (j / C::kStages) & 1, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(bar(C::kBarPFull + bj), (j >> 1) & 1, abort_flag)) return false;
+        if (!mbar_wait(bar(C::kBarVFull + s), (j / C::kStages) & 1, abort_flag)) return false;
         tc_fence_after();
         const uint32_t vbase = base + C::kVOff + s * C::kTileBytes;
         const uint32_t pcol = bj ? C::kColP1 : C::kColP0;
@@ -274,9 +222,27 @@ __global__ void __launch_bounds__(320, 1) attn_qbsa_kernel(const __grid_constant
         }
         mma_commit(bar(C::kBarPVDone));
         mma_commit(bar(C::kBarVEmpty + s));
-        mma_commit(bar(C::kBarPFree + bj));
+        return true;
+      };
+      const uint32_t qbase = base + C::kQOff;
+      for (int it = 0; ok && it < n; ++it) {
+        const int s = it % C::kStages;
+        const int bi = it & 1;
+        if (!mbar_wait(bar(C::kBarKFull + s), (it / C::kStages) & 1, abort_flag)) { ok = false; break; }
+        if (it >= 2 && !mbar_wait(bar(C::kBarSFree + bi), ((it - 2) >> 1) & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t kbase = base + C::kKOff + s * C::kTileBytes;
+        const uint32_t scol = bi ? C::kColS1 : C::kColS0;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          mma_i8_ss(tmem + scol, sdesc_sw128(qbase + kk * 32, 16, 1024), sdesc_sw128(kbase + kk * 32, 16, 1024),
+                    idesc_qk, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(bar(C::kBarSFull + bi));
+        mma_commit(bar(C::kBarKEmpty + s));
+        if (it >= 1 && !issue_pv(it - 1)) { ok = false; break; }
       }
-      if (ok) mma_commit(bar(C::kBarOFinal));
+      if (ok && issue_pv(n - 1)) mma_commit(bar(C::kBarOFinal));
     }
   } else {
     // ---------------------------------------------------------------- softmax warps
@@ -289,130 +255,76 @@ __global__ void __launch_bounds__(320, 1) attn_qbsa_kernel(const __grid_constant
     const uint32_t o_col = tmem + lane_off + C::kColO + half * 64;
     const uint32_t l_col = tmem + lane_off + C::kColL;
 
-    // columns of step i that lie inside S_kv, in this half
-    auto valid_cols = [&](int i) -> int { return min(kTile, p.Skv - static_cast<int>(list[i]) * kTile) - half * 64; };
-    auto s_addr = [&](int i) -> uint32_t { return tmem + lane_off + ((i & 1) ? C::kColS1 : C::kColS0) + half * 64; };
-    auto mask_tail = [&](int i, uint32_t (&r)[64]) {
-      const int valid = valid_cols(i);
-      if (valid < 64) {
-#pragma unroll
-        for (int x = 0; x < 64; ++x)
-          if (x >= valid) r[x] = 0x80000000u;  // INT32_MIN: below every real dot product
-      }
-    };
-    // the paired warp's partial row max of step i (both halves published theirs first)
-    auto publish_max = [&](int i, int32_t pmax) { xch[(i & 1) * 256 + half * 128 + row] = pmax; };
-    auto combine_max = [&](int i, int32_t pmax) -> int32_t {
-      qbsa_named_bar_sync(1 + quarter, 64);
-      return max(pmax, xch[(i & 1) * 256 + (half ^ 1) * 128 + row]);
-    };
-
     float m = kNegInf;    // running max, log2 domain
     float ref = kNegInf;  // power-of-two reference of the FP8 weights (an integer)
-    float resc = 1.0f;    // pending exact O / L rescale for the current step
     bool ok = true;
-    // decide the reference for step i from its row max; sets the pending rescale
-    auto step_ref = [&](int i, int32_t tmax) {
+    for (int it = 0; it < n; ++it) {
+      const int kb = list[it];
+      const int bi = it & 1;
+      const float cst = cst_list[it];
+      const int valid = min(kTile, p.Skv - kb * kTile) - half * 64;  // valid columns of this half
+      // never leave the loop early (the paired warp waits on named barriers below)
+      if (ok) ok = mbar_wait(bar(C::kBarSFull + bi), (it >> 1) & 1, abort_flag);
+      tc_fence_after();
+      float sv[64];  // exact: |dot| <= 128 * 127^2 < 2^24
+      {
+        uint32_t r[64];
+        tmem_ld64_wait(tmem + lane_off + (bi ? C::kColS1 : C::kColS0) + half * 64, r);
+#pragma unroll
+        for (int x = 0; x < 64; ++x) sv[x] = __int2float_rn(static_cast<int32_t>(r[x]));
+      }
+      tc_fence_before();
+      mbar_arrive(bar(C::kBarSFree + bi));
+
+      if (valid < 64) {  // tail block: keys past S_kv get -inf (p = 0 below)
+#pragma unroll
+        for (int x = 0; x < 64; ++x)
+          if (x >= valid) sv[x] = kNegInf;
+      }
+      const float pmax = max64(sv);
+      float* slot = xch + (it & 1) * 256;
+      slot[half * 128 + row] = pmax;
+      qbsa_named_bar_sync(1 + quarter, 64);
+      const float tmax = fmaxf(pmax, slot[(half ^ 1) * 128 + row]);
+
       // max(t) * c == max(t * c): multiplication by c > 0 is monotone in float
-      m = fmaxf(m, __int2float_rn(tmax) * cst_list[i]);
-      // re-set to ceil(m) once m exceeds it by more than 8: p <= 2^8 < 448, exact rescales
+      const float m_blk = tmax * cst;
+      m = fmaxf(m, m_blk);
+      // power-of-two reference: re-set to ceil(m) once m exceeds it by more than 8, so
+      // p <= 2^8 stays below E4M3's 448 and every rescale is an exact power of two
       const bool upd = (ref == kNegInf) || (m > ref + 8.0f);
       const float new_ref = upd ? ceilf(m) : ref;
-      if (upd && ref != kNegInf) {
-        const int dexp = static_cast<int>(ref - new_ref);  // 2^dexp from its exponent bits
-        resc = (dexp < -126) ? 0.f : __int_as_float((127 + dexp) << 23);
-      } else {
-        resc = 1.0f;
-      }
+      const bool need = upd && (ref != kNegInf);
+      // 2^(ref - new_ref) built from its exponent bits (exact; flush below 2^-126)
+      const int dexp = need ? static_cast<int>(ref - new_ref) : 0;
+      const float a = (dexp < -126) ? 0.f : __int_as_float((127 + dexp) << 23);
       ref = new_ref;
-    };
-    uint32_t ra[64], rb[64];  // raw S of the current and the next step
-    if (n > 0) {
-      if (ok) ok = mbar_wait(bar(C::kBarSFull), 0, abort_flag);
-      tc_fence_after();
-      tmem_ld64_issue(s_addr(0), ra);
-      tmem_ld64_wait(ra);
-      tc_fence_before();
-      mbar_arrive(bar(C::kBarSFree));
-      mask_tail(0, ra);
-      const int32_t pm = imax64(ra);
-      publish_max(0, pm);
-      step_ref(0, combine_max(0, pm));
-    }
-    // One step: weights of step it from rc, while S(it+1) streams into rn.  Never leaves
-    // early: the paired warp waits on the named barrier in combine_max.
-    // E4M3 weights of the 32 columns [c0, c0+32) of step it, stored to its P buffer
-    auto weights32 = [&](int it, const uint32_t (&rc)[64], int c0, float cst, int valid) {
-      uint32_t pk[8];
-#pragma unroll
-      for (int x = 0; x < 8; ++x) {
-        const int e = c0 + 4 * x;
-        pk[x] = pack_e4m3x4(ex2(fmaf(__int2float_rn(static_cast<int32_t>(rc[e])), cst, -ref)),
-                            ex2(fmaf(__int2float_rn(static_cast<int32_t>(rc[e + 1])), cst, -ref)),
-                            ex2(fmaf(__int2float_rn(static_cast<int32_t>(rc[e + 2])), cst, -ref)),
-                            ex2(fmaf(__int2float_rn(static_cast<int32_t>(rc[e + 3])), cst, -ref)));
-        if (valid < 64) {  // keys past S_kv weigh exactly 0
-          uint32_t keep = 0;
-#pragma unroll
-          for (int y = 0; y < 4; ++y)
-            if (e + y < valid) keep |= 0xFFu << (8 * y);
-          pk[x] &= keep;
-        }
-      }
-      tmem_st8(tmem + lane_off + ((it & 1) ? C::kColP1 : C::kColP0) + half * 16 + c0 / 4, pk);
-    };
-    auto step = [&](int it, uint32_t (&rc)[64], uint32_t (&rn)[64]) {
-      const bool has_next = it + 1 < n;
-      // P buffer it & 1 was read by P·V(it-2)
-      if (it >= 2 && ok) ok = mbar_wait(bar(C::kBarPFree + (it & 1)), ((it - 2) >> 1) & 1, abort_flag);
-      tc_fence_after();
-      const float cst = cst_list[it];
-      const int valid = valid_cols(it);
-      weights32(it, rc, 0, cst, valid);
-      if (has_next) {
-        if (ok) ok = mbar_wait(bar(C::kBarSFull + ((it + 1) & 1)), ((it + 1) >> 1) & 1, abort_flag);
-        tc_fence_after();
-        tmem_ld64_issue(s_addr(it + 1), rn);  // completes while the second half is computed
-      }
-      weights32(it, rc, 32, cst, valid);
-      if (has_next) {
-        tmem_ld64_wait(rn);
-        tc_fence_before();
-        mbar_arrive(bar(C::kBarSFree + ((it + 1) & 1)));
-        mask_tail(it + 1, rn);
-      } else {
-#pragma unroll
-        for (int x = 0; x < 64; ++x) rn[x] = 0x80000000u;
-      }
-      const int32_t pmax_next = imax64(rn);
-      if (has_next) publish_max(it + 1, pmax_next);
-      // pending rescale of O and L (reference moved at this step): after P·V(it-1)
-      if (__any_sync(0xffffffffu, resc != 1.0f)) {
+      if (__any_sync(0xffffffffu, need)) {
         if (ok) ok = mbar_wait(bar(C::kBarPVDone), (it - 1) & 1, abort_flag);
         tc_fence_after();
-        uint32_t o[32];
-#pragma unroll 1
-        for (int ch = 0; ch < 2; ++ch) {
-          tmem_ld32_wait(o_col + ch * 32, o);
+        uint32_t r[32];
 #pragma unroll
-          for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * resc);
-          tmem_st32(o_col + ch * 32, o);
-          tmem_st_wait();
+        for (int ch = 0; ch < 2; ++ch) {
+          tmem_ld32_wait(o_col + ch * 32, r);
+#pragma unroll
+          for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(__uint_as_float(r[x]) * a);
+          tmem_st32(o_col + ch * 32, r);
         }
-        if (half == 0) tmem_st1(l_col, __float_as_uint(__uint_as_float(tmem_ld1_wait(l_col)) * resc));
+        if (half == 0) tmem_st1(l_col, __float_as_uint(__uint_as_float(tmem_ld1_wait(l_col)) * a));
         tmem_st_wait();
       }
-      tmem_st_wait();  // both halves of P(it) are in TMEM
-      tc_fence_before();
-      mbar_arrive(bar(C::kBarPFull + (it & 1)));
-      if (has_next) step_ref(it + 1, combine_max(it + 1, pmax_next));
-    };
-    // (a register copy per step: unrolling by two to alternate the arrays spills registers,
-    // and the asynchronously loaded array must never be spilled before its wait)
-    for (int it = 0; it < n; ++it) {
-      step(it, ra, rb);
+      // p = 2^(t c - R) held in FP16 (the precision of P before its FP8 rounding),
+      // two weights per ex2, then rounded to E4M3
+      uint32_t pk[16];
 #pragma unroll
-      for (int x = 0; x < 64; ++x) ra[x] = rb[x];
+      for (int x = 0; x < 16; ++x) {
+        pk[x] = exp2_e4m3x4(fmaf(sv[4 * x], cst, -ref), fmaf(sv[4 * x + 1], cst, -ref),
+                            fmaf(sv[4 * x + 2], cst, -ref), fmaf(sv[4 * x + 3], cst, -ref));
+      }
+      tmem_st16(tmem + lane_off + (bi ? C::kColP1 : C::kColP0) + half * 16, pk);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar(C::kBarPFull + bi));
     }
 
     // ------------------------------------------------------------ epilogue
