@@ -178,13 +178,25 @@ def time_steps(fn, steps: int, warmup: int, stream, dist=None, sampler=None):
     return total, per, clocks
 
 
-def max_over_ranks(x: float, dist):
+def max_over_ranks(x: float, dist, device="cuda"):
+    """The largest value of x over all ranks (x itself without a process group)."""
     if dist is None:
         return x
     import torch
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def weak_scaling_value(local_total_ms: float, flops_per_step: float, steps: int, dist, device="cuda"):
+    """(max-over-ranks time of the timed span in ms, whole-job TFLOP/s).
+
+    Every rank runs the same per-GPU workload, so the job's work is world x steps x
+    flops_per_step, delivered in the slowest rank's time.
+    """
+    world = 1 if dist is None else dist.get_world_size()
+    span_ms = max_over_ranks(local_total_ms, dist, device)
+    return span_ms, world * flops_per_step * steps / (span_ms / 1e3) / 1e12
 
 
 def cpu_oracle_sample(inp_host, n_qblocks: int):
@@ -306,9 +318,8 @@ def run_ours(args):
     sampler = ClockSampler(local)
     total_ms, per_ms, clocks = time_steps(step, args.steps, args.warmup, stream, dist, sampler)
     qb.check(device)
-    total_ms = max_over_ranks(total_ms, dist)
+    total_ms, value = weak_scaling_value(total_ms, executed, args.steps, dist)
     ms_step = total_ms / args.steps
-    value = world * executed * args.steps / (total_ms / 1e3) / 1e12
     launch_ms = sum(per_ms) / len(per_ms)
     achieved = executed / (launch_ms / 1e3) / 1e12
 
