@@ -379,17 +379,19 @@ __device__ __forceinline__ uint32_t pack_e4m3x4(float a0, float a1, float a2, fl
   return r;
 }
 
-// Four exponents x (log2 units) -> 2^x held in FP16 (ex2 on f16x2, two per
-// instruction) -> four E4M3 bytes (byte i = value i), nearest even, saturating.
+// Four exponents x (log2 units) -> 2^x (fp32 ex2) rounded to FP16 -> four E4M3 bytes
+// (byte i = value i); both roundings nearest even, the second saturating.
 __device__ __forceinline__ uint32_t exp2_e4m3x4(float x0, float x1, float x2, float x3) {
   uint32_t r;
-  asm("{\n\t.reg .b32 h01, h23, e01, e23;\n\t.reg .b16 lo, hi;\n\t"
-      "cvt.rn.f16x2.f32 h01, %2, %1;\n\t"
-      "cvt.rn.f16x2.f32 h23, %4, %3;\n\t"
-      "ex2.approx.f16x2 e01, h01;\n\t"
-      "ex2.approx.f16x2 e23, h23;\n\t"
-      "cvt.rn.satfinite.e4m3x2.f16x2 lo, e01;\n\t"
-      "cvt.rn.satfinite.e4m3x2.f16x2 hi, e23;\n\t"
+  asm("{\n\t.reg .f32 e0, e1, e2, e3;\n\t.reg .b32 h01, h23;\n\t.reg .b16 lo, hi;\n\t"
+      "ex2.approx.ftz.f32 e0, %1;\n\t"
+      "ex2.approx.ftz.f32 e1, %2;\n\t"
+      "ex2.approx.ftz.f32 e2, %3;\n\t"
+      "ex2.approx.ftz.f32 e3, %4;\n\t"
+      "cvt.rn.f16x2.f32 h01, e1, e0;\n\t"
+      "cvt.rn.f16x2.f32 h23, e3, e2;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f16x2 lo, h01;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f16x2 hi, h23;\n\t"
       "mov.b32 %0, {lo, hi};\n\t}"
       : "=r"(r)
       : "f"(x0), "f"(x1), "f"(x2), "f"(x3));
