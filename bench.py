@@ -370,6 +370,9 @@ def run_ours(args):
                                 "sample": desc + f", {secs:.1f} s"}
 
     extra = {}
+    # ---------------------------------------------------------------- bf16 block-sparse, same mask
+    if not args.no_dense:
+        extra["bsa_bf16_same_mask"] = bsa_line(device, stream, inp, executed, bf16_peak, ms_step)
     del inp
     torch.cuda.empty_cache()
     # ---------------------------------------------------------------- dense bf16 video workload
@@ -407,6 +410,30 @@ def qbsa_line(device, stream, S, keep, fp8_peak):
     torch.cuda.empty_cache()
     return {"S": S, "keep": keep, "ms": ms, "executed_tflops": executed / ms / 1e9,
             "dense_equivalent_tflops": dense_eq / ms / 1e9, "pct_of_fp8_peak": 100 * executed / ms / 1e9 / fp8_peak}
+
+
+def bsa_line(device, stream, inp, executed, bf16_peak, qbsa_ms):
+    """bf16 block-sparse attention on the quantized workload's shape and block mask."""
+    import torch
+    import quantized_block_sparse_attn_b200 as qb
+    from workloads import CONFIGS, device_blocky_qk_bf16, device_iid_normal_bf16
+    N, S, D, seed = inp["N"], inp["S"], inp["D"], inp["seed"]
+    q = device_blocky_qk_bf16(seed, "q", 1, N, S, D, device)
+    k = device_blocky_qk_bf16(seed, "k", 1, N, S, D, device)
+    v = device_iid_normal_bf16(seed, 2, (1, N, S, D), device)
+    out = torch.empty_like(q)
+
+    def step():
+        qb.bsa_fwd(q, k, v, inp["bm"], inp["scale"], out=out, return_stats=False)
+
+    total, per, _ = time_steps(step, 5, 2, stream)
+    qb.check(device)
+    ms = total / 5
+    del q, k, v, out
+    torch.cuda.empty_cache()
+    return {"workload": f"bsa_fwd bf16 B=1 N=40 S={S} D=128, same block mask", "ms": ms,
+            "executed_tflops": executed / ms / 1e9, "pct_of_bf16_peak": 100 * executed / ms / 1e9 / bf16_peak,
+            "qbsa_speedup_over_bsa": ms / qbsa_ms, "kernel": "attn_dense_kernel<128> (block-mask list)"}
 
 
 def dense_line(device, stream, S, warmup, steps, bf16_peak, dist):

@@ -96,6 +96,22 @@ qbsa_status attn_fwd(const void* q, const void* k, const void* v, int B, int Nq,
                      void* stream);
 
 /*
+ * bsa_fwd -- bf16 block-sparse attention: attn_fwd (BNSD, sparse_mode 0, no atten_mask,
+ * no pse) computed only over the 128x128 blocks kept by block_mask.  This is the BF16
+ * block-sparse baseline ("BSA") that [QBSA] "EagleQBSA单算子性能验证分析" compares the
+ * quantized operator with, on the same block mask.
+ *
+ * q, k, v        bf16 BNSD device tensors as in attn_fwd.
+ * block_mask     uint8 [B, Nq, ceil(Sq/128), ceil(Skv/128)], 1 = compute the block;
+ *                ceil(Skv/128) <= 2048.  Keys of blocks not kept are masked; a row with
+ *                no kept block gets out = 0, max = -inf, sum = 0.
+ * Other arguments and outputs as in attn_fwd.
+ */
+qbsa_status bsa_fwd(const void* q, const void* k, const void* v, const uint8_t* block_mask, int B, int Nq, int Nkv,
+                    int Sq, int Skv, int D, float scale, void* attention_out, float* softmax_max, float* softmax_sum,
+                    void* stream);
+
+/*
  * qbsa_fwd -- quantized block-sparse attention forward, [QBSA] "MindIE SD调用方式" and
  * "EagleQBSA量化叠加稀疏方案设计": INT8 Q·Kᵀ with per-128-token-block scales, online
  * softmax, P rounded to FP8 E4M3 (nearest even), FP8 P·V with per-channel V scales,

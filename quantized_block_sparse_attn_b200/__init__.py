@@ -10,6 +10,7 @@ from ._binding import (  # noqa: F401
     QbsaError,
     attn_fwd,
     attn_tile_schedule,
+    bsa_fwd,
     block_lists,
     check,
     lib,

@@ -28,6 +28,7 @@ SIGNATURES = {
     "attn_fwd": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _I, _P, _I, _F, _F, _I, _I64, _I64,
                       _P, _P, _P, _P, _P, _P]),
     "qbsa_fwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P]),
+    "bsa_fwd": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P]),
     "qbsa_quantize_qk": (_I, [_P, _I, _I, _I, _I, _P, _P, _P]),
     "qbsa_quantize_v": (_I, [_P, _I, _I, _I, _I, _P, _P, _P]),
     "attn_tile_schedule": (_I, [_I64, _I64, _I, _I64, _I64, _P, _P, _P, _P, _I64]),
@@ -141,6 +142,29 @@ def attn_fwd(q, k, v, head_num: int, input_layout: str = "BNSD", *, atten_mask=N
                    next_tokens, None if cq is None else cq.ctypes.data_as(ctypes.c_void_p),
                    None if ck is None else ck.ctypes.data_as(ctypes.c_void_p), _ptr(out), _ptr(softmax_max),
                    _ptr(softmax_sum), _stream(dev)))
+    if host:
+        return tuple(None if t is None else t.cpu() for t in (out, softmax_max, softmax_sum))
+    return out, softmax_max, softmax_sum
+
+
+def bsa_fwd(q, k, v, block_mask, scale: float, *, out=None, softmax_max=None, softmax_sum=None,
+            return_stats: bool = True, device=None):
+    """bf16 block-sparse attention (BNSD): attn_fwd over the 128x128 blocks kept by block_mask."""
+    import torch
+    host = not q.is_cuda
+    dev = torch.device(device or (q.device if q.is_cuda else "cuda:0"))
+    q, k, v, block_mask = _on_cuda([q, k, v, block_mask], dev)
+    B, Nq, Sq, D = q.shape
+    Nkv, Skv = k.shape[1], k.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    if return_stats:
+        if softmax_max is None:
+            softmax_max = torch.empty((B, Nq, Sq), dtype=torch.float32, device=dev)
+        if softmax_sum is None:
+            softmax_sum = torch.empty((B, Nq, Sq), dtype=torch.float32, device=dev)
+    _ck(lib().bsa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(block_mask), B, Nq, Nkv, Sq, Skv, D, scale, _ptr(out),
+                      _ptr(softmax_max), _ptr(softmax_sum), _stream(dev)))
     if host:
         return tuple(None if t is None else t.cpu() for t in (out, softmax_max, softmax_sum))
     return out, softmax_max, softmax_sum

@@ -56,6 +56,9 @@ struct DenseParams {
   int n_qtiles;   // BNSD/BSND: ceil(Sq/128)
   int n_rank;     // query tiles per head (all batches / sequences)
   int head_grp;   // query heads per L2 group
+  // optional 128x128 block mask [B, Nq, n_qtiles, mask_nkb] (1 = compute), BNSD / BSND only
+  const uint8_t* block_mask;
+  int mask_nkb;
   float scale;
   // TND tables (sequences in processing order)
   int n_seq;
@@ -75,7 +78,9 @@ struct DenseCfg {
   static constexpr int kKOff = kQOff + kTileBytes;
   static constexpr int kVOff = kKOff + kStages * kTileBytes;
   static constexpr int kXOff = kVOff + kStages * kTileBytes;  // row-max exchange: float [2][2][128]
-  static constexpr int kBarOff = kXOff + 2 * 2 * 128 * 4;
+  static constexpr int kListOff = kXOff + 2 * 2 * 128 * 4;    // uint16 kept K tiles (block mask)
+  static constexpr int kMaxListed = 2048;
+  static constexpr int kBarOff = kListOff + kMaxListed * 2;
   // barriers
   static constexpr int kBarQFull = 0;
   static constexpr int kBarKFull = 1;
@@ -172,9 +177,23 @@ __global__ void __launch_bounds__(320, 1) attn_dense_kernel(const __grid_constan
   const int g = w.h / p.group;
   const Band band = band_of(p.sparse_mode, p.pre_tokens, p.next_tokens, w.sq, w.skv);
   const TileRange tr = tile_range(w.qt, w.sq, w.skv, band);
-  const int n = tr.kt_end - tr.kt_begin;
   const bool general_mask = (p.atten_mask != nullptr) || (p.pse != nullptr);
+  uint16_t* klist = reinterpret_cast<uint16_t*>(smem + C::kListOff);
+  int* count_slot = reinterpret_cast<int*>(smem + C::kMiscOff + 8);
 
+  if (p.block_mask != nullptr && warp == 0) {
+    // kept K tiles of this query tile inside its band range, ascending
+    const uint8_t* mrow = p.block_mask + (((int64_t)w.b * p.Nq + w.h) * p.n_qtiles + w.qt) * p.mask_nkb;
+    int cnt = 0;
+    for (int j0 = tr.kt_begin; j0 < tr.kt_end; j0 += 32) {
+      const int j = j0 + lane;
+      const bool keep = (j < tr.kt_end) && (mrow[j] != 0);
+      const uint32_t bal = __ballot_sync(0xffffffffu, keep);
+      if (keep) klist[cnt + __popc(bal & ((1u << lane) - 1u))] = static_cast<uint16_t>(j);
+      cnt += __popc(bal);
+    }
+    if (lane == 0) *count_slot = cnt;
+  }
   if (threadIdx.x == 0) {
     *abort_flag = 0;
     mbar_init(bar(C::kBarQFull), 1);
@@ -204,6 +223,9 @@ __global__ void __launch_bounds__(320, 1) attn_dense_kernel(const __grid_constan
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  const bool listed = p.block_mask != nullptr;
+  const int n = listed ? *count_slot : tr.kt_end - tr.kt_begin;
+  auto ktile = [&](int it) -> int { return listed ? static_cast<int>(klist[it]) : tr.kt_begin + it; };
 
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
@@ -218,7 +240,7 @@ __global__ void __launch_bounds__(320, 1) attn_dense_kernel(const __grid_constan
       for (int it = 0; it < n; ++it) {
         const int s = it % C::kStages;
         const uint32_t ph = (it / C::kStages) & 1;
-        const int kv_row = static_cast<int>(w.kv_row0 + (int64_t)(tr.kt_begin + it) * kTile);
+        const int kv_row = static_cast<int>(w.kv_row0 + (int64_t)ktile(it) * kTile);
         if (it >= C::kStages && !mbar_wait(bar(C::kBarKEmpty + s), ph ^ 1, abort_flag)) break;
         mbar_arrive_expect_tx(bar(C::kBarKFull + s), C::kTileBytes);
         for (int sub = 0; sub < D / 64; ++sub)
@@ -302,7 +324,7 @@ __global__ void __launch_bounds__(320, 1) attn_dense_kernel(const __grid_constan
     float m_ref = kNegInf, m_true = kNegInf, l = 0.f;  // l: this half's partial sum
     bool ok = true;
     for (int it = 0; it < n; ++it) {
-      const int kt = tr.kt_begin + it;
+      const int kt = ktile(it);
       const int bi = it & 1;
       // never leave the loop early: the paired warp waits on named barriers below, so
       // after a failed (timed-out) wait the remaining iterations run without waiting

@@ -126,12 +126,14 @@ int qbsa_version(void) { return 100; }
 
 const char* qbsa_last_error(void) { return g_last_error.c_str(); }
 
-qbsa_status attn_fwd(const void* q, const void* k, const void* v, int B, int Nq, int Nkv, int Sq, int Skv, int D,
-                     int head_num, qbsa_layout input_layout, const uint8_t* atten_mask, qbsa_mask_shape mask_shape,
-                     const void* pse, int pse_batch_bcast, float scale, float keep_prob, int sparse_mode,
-                     int64_t pre_tokens, int64_t next_tokens, const int64_t* actual_seq_qlen,
-                     const int64_t* actual_seq_kvlen, void* attention_out, float* softmax_max, float* softmax_sum,
-                     void* stream) {
+// attn_fwd, optionally restricted to the 128x128 blocks kept by block_mask (bsa_fwd).
+static qbsa_status attn_fwd_impl(const void* q, const void* k, const void* v, int B, int Nq, int Nkv, int Sq, int Skv,
+                                 int D, int head_num, qbsa_layout input_layout, const uint8_t* atten_mask,
+                                 qbsa_mask_shape mask_shape, const void* pse, int pse_batch_bcast, float scale,
+                                 float keep_prob, int sparse_mode, int64_t pre_tokens, int64_t next_tokens,
+                                 const int64_t* actual_seq_qlen, const int64_t* actual_seq_kvlen,
+                                 void* attention_out, float* softmax_max, float* softmax_sum, void* stream,
+                                 const uint8_t* block_mask) {
   // ---------------------------------------------------------------- validation
   if (!q || !k || !v || !attention_out) return fail(QBSA_ERR_INVALID, "q, k, v and attention_out must be non-null");
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(attention_out))
@@ -284,8 +286,34 @@ qbsa_status attn_fwd(const void* q, const void* k, const void* v, int B, int Nq,
   if ((st = make_map(&prm.tm_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, k, kd, ks, 64)) != QBSA_OK) return st;
   if ((st = make_map(&prm.tm_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, v, kd, ks, 64)) != QBSA_OK) return st;
 
+  if (block_mask) {
+    prm.block_mask = block_mask;
+    prm.mask_nkb = (Skv + qbsa::kTile - 1) / qbsa::kTile;
+  }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return D == 128 ? launch_dense<128>(prm, n_work, s) : launch_dense<64>(prm, n_work, s);
+}
+
+qbsa_status attn_fwd(const void* q, const void* k, const void* v, int B, int Nq, int Nkv, int Sq, int Skv, int D,
+                     int head_num, qbsa_layout input_layout, const uint8_t* atten_mask, qbsa_mask_shape mask_shape,
+                     const void* pse, int pse_batch_bcast, float scale, float keep_prob, int sparse_mode,
+                     int64_t pre_tokens, int64_t next_tokens, const int64_t* actual_seq_qlen,
+                     const int64_t* actual_seq_kvlen, void* attention_out, float* softmax_max, float* softmax_sum,
+                     void* stream) {
+  return attn_fwd_impl(q, k, v, B, Nq, Nkv, Sq, Skv, D, head_num, input_layout, atten_mask, mask_shape, pse,
+                       pse_batch_bcast, scale, keep_prob, sparse_mode, pre_tokens, next_tokens, actual_seq_qlen,
+                       actual_seq_kvlen, attention_out, softmax_max, softmax_sum, stream, nullptr);
+}
+
+qbsa_status bsa_fwd(const void* q, const void* k, const void* v, const uint8_t* block_mask, int B, int Nq, int Nkv,
+                    int Sq, int Skv, int D, float scale, void* attention_out, float* softmax_max, float* softmax_sum,
+                    void* stream) {
+  if (!block_mask) return fail(QBSA_ERR_INVALID, "bsa_fwd needs a block_mask");
+  if ((Skv + qbsa::kTile - 1) / qbsa::kTile > qbsa::DenseCfg<128>::kMaxListed)
+    return fail(QBSA_ERR_UNSUPPORTED, "ceil(Skv/128) exceeds %d", qbsa::DenseCfg<128>::kMaxListed);
+  return attn_fwd_impl(q, k, v, B, Nq, Nkv, Sq, Skv, D, Nq, QBSA_LAYOUT_BNSD, nullptr, QBSA_MASK_NONE, nullptr, 0,
+                       scale, 1.0f, 0, INT64_C(2147483647), INT64_C(2147483647), nullptr, nullptr, attention_out,
+                       softmax_max, softmax_sum, stream, block_mask);
 }
 
 // ------------------------------------------------------------------------------

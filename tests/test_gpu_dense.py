@@ -158,3 +158,21 @@ def test_video_workload_sampled():
     v = iid_normal_bf16(c["seed"], 2, 1, N, S, D)
     rows = np.concatenate([np.arange(b * 128, b * 128 + 128) for b in sample_rows(c["seed"], S, 4)])
     _run_and_compare(q, k, v, "BNSD", N, c["scale"], 0, q_rows=rows, heads=[(0, h) for h in heads])
+
+
+@pytest.mark.parametrize("B,Nq,Nkv,S,D,keep", [(1, 2, 1, 300, 128, 0.5), (2, 2, 2, 1024, 64, 0.25),
+                                               (1, 3, 1, 640, 128, 1.0)])
+def test_bsa_parity(B, Nq, Nkv, S, D, keep):
+    """bf16 block-sparse attention = the dense oracle with the unkept blocks masked."""
+    from workloads import block_keep_mask
+    q, k, v = _bnsd(12, B, Nq, Nkv, S, S, D)
+    nb = -(-S // 128)
+    bm = block_keep_mask(12, B, Nq, nb, nb, keep)
+    bm[0, 0, 1 % nb, :] = 0  # one query tile with no kept block
+    out, smax, ssum = qb.bsa_fwd(dev_bf16(q), dev_bf16(k), dev_bf16(v), dev(bm), D ** -0.5)
+    qb.check()
+    el = np.repeat(np.repeat(bm, 128, axis=2), 128, axis=3)[:, :, :S, :S]
+    ref, rmax, rsum = dense.attention_forward(q, k, v, layout="BNSD", scale=D ** -0.5,
+                                              atten_mask=(el == 0).astype(np.uint8))
+    compare_out(host_f64(out), ref, DENSE_MAX_ABS, DENSE_MEAN_ABS)
+    compare_stats(smax.cpu().numpy(), ssum.cpu().numpy(), rmax, rsum)
