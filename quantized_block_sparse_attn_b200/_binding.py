@@ -87,6 +87,38 @@ def _on_cuda(tensors, device):
     return out
 
 
+def _split_outputs(host, outs):
+    """In host mode, caller-given output tensors on the host become copy destinations and the kernel writes
+    fresh device buffers; otherwise every given output must already be a device tensor."""
+    dev_outs, dsts = [], []
+    for t in outs:
+        if t is not None and not t.is_cuda:
+            if not host:
+                raise ValueError("output tensors must be on the GPU when the inputs are")
+            dev_outs.append(None)
+            dsts.append(t)
+        else:
+            dev_outs.append(t)
+            dsts.append(None)
+    return dev_outs, dsts
+
+
+def _to_host(results, dsts, device):
+    """Copy device results into pinned host tensors (the caller's or new ones); waits for the copies."""
+    import torch
+    res = []
+    for t, dst in zip(results, dsts):
+        if t is None:
+            res.append(None)
+            continue
+        if dst is None:
+            dst = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+        dst.copy_(t, non_blocking=True)
+        res.append(dst)
+    torch.cuda.current_stream(device).synchronize()
+    return tuple(res)
+
+
 def attn_fwd(q, k, v, head_num: int, input_layout: str = "BNSD", *, atten_mask=None, mask_shape=None, pse=None,
              scale: float = 1.0, keep_prob: float = 1.0, sparse_mode: int = 0, pre_tokens: int = INF_TOKENS,
              next_tokens: int = INF_TOKENS, actual_seq_qlen=None, actual_seq_kvlen=None, out=None,
@@ -100,6 +132,7 @@ def attn_fwd(q, k, v, head_num: int, input_layout: str = "BNSD", *, atten_mask=N
     host = not q.is_cuda
     dev = torch.device(device or (q.device if q.is_cuda else "cuda:0"))
     q, k, v, atten_mask, pse = _on_cuda([q, k, v, atten_mask, pse], dev)
+    (out, softmax_max, softmax_sum), dsts = _split_outputs(host, (out, softmax_max, softmax_sum))
     for t in (q, k, v):
         if t.dtype != torch.bfloat16 or not t.is_contiguous():
             raise ValueError("q, k, v must be contiguous bfloat16 tensors")
@@ -143,7 +176,7 @@ def attn_fwd(q, k, v, head_num: int, input_layout: str = "BNSD", *, atten_mask=N
                    None if ck is None else ck.ctypes.data_as(ctypes.c_void_p), _ptr(out), _ptr(softmax_max),
                    _ptr(softmax_sum), _stream(dev)))
     if host:
-        return tuple(None if t is None else t.cpu() for t in (out, softmax_max, softmax_sum))
+        return _to_host((out, softmax_max, softmax_sum), dsts, dev)
     return out, softmax_max, softmax_sum
 
 
@@ -154,6 +187,7 @@ def bsa_fwd(q, k, v, block_mask, scale: float, *, out=None, softmax_max=None, so
     host = not q.is_cuda
     dev = torch.device(device or (q.device if q.is_cuda else "cuda:0"))
     q, k, v, block_mask = _on_cuda([q, k, v, block_mask], dev)
+    (out, softmax_max, softmax_sum), dsts = _split_outputs(host, (out, softmax_max, softmax_sum))
     B, Nq, Sq, D = q.shape
     Nkv, Skv = k.shape[1], k.shape[2]
     if out is None:
@@ -166,7 +200,7 @@ def bsa_fwd(q, k, v, block_mask, scale: float, *, out=None, softmax_max=None, so
     _ck(lib().bsa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(block_mask), B, Nq, Nkv, Sq, Skv, D, scale, _ptr(out),
                       _ptr(softmax_max), _ptr(softmax_sum), _stream(dev)))
     if host:
-        return tuple(None if t is None else t.cpu() for t in (out, softmax_max, softmax_sum))
+        return _to_host((out, softmax_max, softmax_sum), dsts, dev)
     return out, softmax_max, softmax_sum
 
 
@@ -178,6 +212,7 @@ def qbsa_fwd(q_i8, k_i8, q_scale, k_scale, v_fp8, v_scale, block_mask, scale: fl
     dev = torch.device(device or (q_i8.device if q_i8.is_cuda else "cuda:0"))
     q_i8, k_i8, q_scale, k_scale, v_fp8, v_scale, block_mask = _on_cuda(
         [q_i8, k_i8, q_scale, k_scale, v_fp8, v_scale, block_mask], dev)
+    (out, softmax_max, softmax_sum), dsts = _split_outputs(host, (out, softmax_max, softmax_sum))
     B, Nq, Sq, D = q_i8.shape
     Nkv, Skv = k_i8.shape[1], k_i8.shape[2]
     if out is None:
@@ -192,7 +227,7 @@ def qbsa_fwd(q_i8, k_i8, q_scale, k_scale, v_fp8, v_scale, block_mask, scale: fl
                    _ptr(block_mask), B, Nq, Nkv, Sq, Skv, D, scale, _ptr(out), _ptr(softmax_max),
                    _ptr(softmax_sum), _stream(dev)))
     if host:
-        return tuple(None if t is None else t.cpu() for t in (out, softmax_max, softmax_sum))
+        return _to_host((out, softmax_max, softmax_sum), dsts, dev)
     return out, softmax_max, softmax_sum
 
 
