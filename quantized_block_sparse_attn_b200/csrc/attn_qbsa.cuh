@@ -7,24 +7,30 @@
 // block-sparse mask are computed (section "背景介绍"; block_sparse_mask and
 // block_shape=[128,128] in section "MindIE SD调用方式").
 //
-// One CTA per (batch, head, 128-row query block).  Warp 0 first compacts the CTA's row
-// of the block mask into the ascending list of kept key blocks in shared memory, with
-// each block's dequantisation constant s_q * s_k * scale * log2(e).  Then:
-//   warp 0      TMA producer (Q once; K and V tiles of kept blocks, 3-stage rings)
-//   warp 1      TMEM owner + MMA issuer: S = Q8 K8ᵀ (kind::i8, s32 in TMEM);
-//               O += P8 V8 (kind::f8f6f4, A = P8 from TMEM, B = V8 MN-major) and
-//               L += P8 · 1 (N = 16 ones matrix), so L is exactly Σ p8.
-//   warps 2..9  softmax: query row 32*(warp%4)+lane; warps 2..5 own key columns [0,64),
-//               warps 6..9 [64,128), exchanging partial row maxima through shared
-//               memory.  Exact s32 -> f32 (|dot| < 2^24), online softmax whose weights
-//               p = 2^(z - R) use a power-of-two reference R re-set to ceil(running max)
-//               only when the max exceeds it by more than 8 (exact power-of-two
-//               rescales of O and L, rare), P -> E4M3 into TMEM, epilogue
+// One CTA per (batch, head, pair of 128-row query blocks).  The two query tiles share
+// the tensor core and take turns on the special-function unit: while one tile's
+// warps load scores and reduce row maxima, the other tile's warps are in their
+// exponentials.  Each tile's row of the block mask is first compacted into the
+// ascending list of kept key blocks in shared memory, with each block's
+// dequantisation constant s_q * s_k * scale * log2(e).  Then:
+//   warps 0..3  softmax of tile 0, warps 4..7 softmax of tile 1: one thread per query
+//               row (TMEM lane 32*(warp%4)+lane), all 128 key columns of a block.
+//               Exact s32 -> f32 (|dot| < 2^24), online softmax whose weights
+//               p = 2^(z - R) use a power-of-two reference R re-set to ceil(running
+//               max) only when the max exceeds it by more than 8 (exact power-of-two
+//               rescales of O and L, rare), P -> FP16 -> E4M3 into TMEM, epilogue
 //               O * v_scale / L -> bf16.
-// TMEM columns: S0 [0,128) S1 [128,256) O [256,384) L [384,400) P0 [448,480) P1 [480,512).
+//   warp 8      TMA producer: Q of both tiles once; K and V tiles of the kept blocks
+//               of both tiles, interleaved (t0 j, t1 j, t0 j+1, ...), 5-stage ring.
+//   warp 9      TMEM owner + MMA issuer, in the order QK0(j), PV0(j-1), QK1(j),
+//               PV1(j-1): S = Q8 K8ᵀ (kind::i8, s32 into the one shared S buffer),
+//               O_t += P8_t V8 (kind::f8f6f4, A = P8 from TMEM, B = V8 MN-major) and
+//               L_t += P8_t · 1 (N = 16 ones matrix), so L is exactly Σ p8.
+// TMEM columns: O0 [0,128) O1 [128,256) S [256,384) P0 [384,416) P1 [416,448)
+//               L0 [448,464) L1 [464,480).
 //
-// CTA order: query heads in groups whose K8/V8 fit in about 48 MB of L2, query blocks
-// in order, heads fastest inside a group.
+// CTA order: query heads in groups whose K8/V8 fit in about 48 MB of L2, query-block
+// pairs in order, heads fastest inside a group.
 #pragma once
 
 #include <cstdint>
@@ -49,41 +55,43 @@ struct QbsaParams {
   float* softmax_max;     // [B, Nq, Sq] or nullptr
   float* softmax_sum;
   int B, Nq, Nkv, Sq, Skv, group, nqb, nkb;
-  int n_rank;             // B * nqb
+  int n_pair;             // ceil(nqb / 2) query-block pairs per (batch, head)
+  int n_rank;             // B * n_pair
   int head_grp;           // query heads per L2 group
   float scale_log2;       // scale * log2(e)
 };
 
 struct QbsaCfg {
   static constexpr int D = 128;
-  static constexpr int kStages = 3;
-  static constexpr int kTileBytes = kTile * 128;  // 128 rows x 128 bytes
-  static constexpr int kQOff = 0;
-  static constexpr int kKOff = kQOff + kTileBytes;
+  static constexpr int kStages = 5;                 // (K, V) tile pairs in flight
+  static constexpr int kTileBytes = kTile * 128;    // 128 rows x 128 bytes
+  static constexpr int kQOff = 0;                   // Q of tile 0, then tile 1
+  static constexpr int kKOff = kQOff + 2 * kTileBytes;
   static constexpr int kVOff = kKOff + kStages * kTileBytes;
-  static constexpr int kOnesOff = kVOff + kStages * kTileBytes;  // 16 x 128 bytes of E4M3 1.0
-  static constexpr int kCOff = kOnesOff + 2048;                   // float dequant constant per kept block
-  static constexpr int kListOff = kCOff + kQbsaMaxKBlocks * 4;    // uint16 kept-block list
-  static constexpr int kXOff = kListOff + kQbsaMaxKBlocks * 2;    // int row-max exchange [2][2][128]
-  static constexpr int kBarOff = kXOff + 2 * 2 * 128 * 4;
+  static constexpr int kOnesOff = kVOff + kStages * kTileBytes;   // 16 x 128 bytes of E4M3 1.0
+  static constexpr int kCOff = kOnesOff + 2048;                    // float [2][kMax] dequant constants
+  static constexpr int kListOff = kCOff + 2 * kQbsaMaxKBlocks * 4;  // uint16 [2][kMax] kept blocks
+  static constexpr int kVscOff = kListOff + 2 * kQbsaMaxKBlocks * 2;  // float [128] value scales
+  static constexpr int kBarOff = kVscOff + 128 * 4;
   static constexpr int kBarQFull = 0;
   static constexpr int kBarKFull = 1;
-  static constexpr int kBarKEmpty = kBarKFull + kStages;
-  static constexpr int kBarVFull = kBarKEmpty + kStages;
-  static constexpr int kBarVEmpty = kBarVFull + kStages;
-  static constexpr int kBarSFull = kBarVEmpty + kStages;
-  static constexpr int kBarSFree = kBarSFull + 2;
-  static constexpr int kBarPFull = kBarSFree + 2;
-  static constexpr int kBarPVDone = kBarPFull + 2;
-  static constexpr int kBarOFinal = kBarPVDone + 1;  // last P·V done (single use)
-  static constexpr int kNumBars = kBarOFinal + 1;
-  static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // tmem addr, abort flag, list count
+  static constexpr int kBarVFull = kBarKFull + kStages;
+  static constexpr int kBarKVEmpty = kBarVFull + kStages;
+  static constexpr int kBarSFull = kBarKVEmpty + kStages;  // [2], per tile
+  static constexpr int kBarSFree = kBarSFull + 2;          // [2], per tile
+  static constexpr int kBarPFull = kBarSFree + 2;          // [2]
+  static constexpr int kBarPVDone = kBarPFull + 2;         // [2]
+  static constexpr int kBarOFinal = kBarPVDone + 2;        // [2], single use
+  static constexpr int kBarDrain = kBarOFinal + 2;         // single use: every MMA retired
+  static constexpr int kNumBars = kBarDrain + 1;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // tmem addr, abort flag, counts[2]
   static constexpr int kSmemBytes = kMiscOff + 16 + 1024;
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256, kColL = 384, kColP0 = 448, kColP1 = 480;
+  static constexpr uint32_t kColO = 0, kColS = 256, kColP = 384, kColL = 448;  // O_t = kColO + 128 t, ...
   static constexpr int kThreads = 320;
-  static constexpr int kSoftmaxThreads = 256;
+  static constexpr int kWarpProducer = 8, kWarpMma = 9;
 };
+static_assert(QbsaCfg::kSmemBytes <= 232448, "shared memory above the 227 KB opt-in limit");
 
 // Compact one row of the block mask (n_kb bytes, 1 = keep) into ascending indices.
 // Executed by one full warp; returns the count (same value in every lane).
@@ -99,8 +107,9 @@ __device__ __forceinline__ int compact_mask_row(const uint8_t* row, int n_kb, ui
   return count;
 }
 
-__device__ __forceinline__ void qbsa_named_bar_sync(int id, int nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+// Every lane waits; the warp proceeds only if all lanes saw the phase complete.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag)) != 0;
 }
 
 __global__ void __launch_bounds__(320, 1) attn_qbsa_kernel(const __grid_constant__ QbsaParams p) {
@@ -116,12 +125,12 @@ __global__ void __launch_bounds__(320, 1) attn_qbsa_kernel(const __grid_constant
   auto bar = [&](int i) -> uint32_t { return bar0 + 8u * static_cast<uint32_t>(i); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
-  int* count_slot = reinterpret_cast<int*>(smem + C::kMiscOff + 8);
-  uint16_t* list = reinterpret_cast<uint16_t*>(smem + C::kListOff);
-  float* cst_list = reinterpret_cast<float*>(smem + C::kCOff);
-  float* xch = reinterpret_cast<float*>(smem + C::kXOff);
+  int* count_slot = reinterpret_cast<int*>(smem + C::kMiscOff + 8);  // [2]
+  uint16_t* lists = reinterpret_cast<uint16_t*>(smem + C::kListOff);
+  float* csts = reinterpret_cast<float*>(smem + C::kCOff);
+  float* vsc = reinterpret_cast<float*>(smem + C::kVscOff);
 
-  // head groups (L2 reuse of K/V), query blocks in order, heads fastest inside a group
+  // head groups (L2 reuse of K/V), query-block pairs in order, heads fastest in a group
   const int64_t per_group = (int64_t)p.head_grp * p.n_rank;
   const int grp = static_cast<int>(blockIdx.x / per_group);
   const int h0 = grp * p.head_grp;
@@ -129,166 +138,221 @@ __global__ void __launch_bounds__(320, 1) attn_qbsa_kernel(const __grid_constant
   const int off = static_cast<int>(blockIdx.x - grp * per_group);
   const int r = off / hcount;
   const int h = h0 + off % hcount;
-  const int qb = r % p.nqb;
-  const int b = r / p.nqb;
+  const int pr = r % p.n_pair;
+  const int b = r / p.n_pair;
   const int g = h / p.group;
 
-  if (warp == 0) {
-    const uint8_t* mrow = p.block_mask + (((int64_t)b * p.Nq + h) * p.nqb + qb) * p.nkb;
-    const int cnt = compact_mask_row(mrow, p.nkb, list, lane);
-    __syncwarp();
-    const float sq = p.q_scale[((int64_t)b * p.Nq + h) * p.nqb + qb];
-    const float* ks = p.k_scale + ((int64_t)b * p.Nkv + g) * p.nkb;
-    for (int i = lane; i < cnt; i += 32) cst_list[i] = (sq * ks[list[i]]) * p.scale_log2;
+  if (warp == 0 || warp == 4) {
+    // kept-block list and dequantisation constants of tile t
+    const int t = warp >> 2;
+    const int qb = 2 * pr + t;
+    uint16_t* list = lists + t * kQbsaMaxKBlocks;
+    int cnt = 0;
+    if (qb < p.nqb) {
+      const uint8_t* mrow = p.block_mask + (((int64_t)b * p.Nq + h) * p.nqb + qb) * p.nkb;
+      cnt = compact_mask_row(mrow, p.nkb, list, lane);
+      __syncwarp();
+      const float sq = p.q_scale[((int64_t)b * p.Nq + h) * p.nqb + qb];
+      const float* ks = p.k_scale + ((int64_t)b * p.Nkv + g) * p.nkb;
+      float* cst = csts + t * kQbsaMaxKBlocks;
+      for (int i = lane; i < cnt; i += 32) cst[i] = (sq * ks[list[i]]) * p.scale_log2;
+    }
+    if (lane == 0) count_slot[t] = cnt;
+  } else if (warp == 1) {
+    // the ones matrix (E4M3 1.0 = 0x38) used to accumulate the row sums of P8
+    uint32_t* ones = reinterpret_cast<uint32_t*>(smem + C::kOnesOff);
+    for (int i = lane; i < 512; i += 32) ones[i] = 0x38383838u;
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  } else if (warp == 2) {
+    const float* vs = p.v_scale + ((int64_t)b * p.Nkv + g) * 128;
+    for (int i = lane; i < 128; i += 32) vsc[i] = vs[i];
+  } else if (warp == C::kWarpProducer) {
     if (lane == 0) {
-      *count_slot = cnt;
       *abort_flag = 0;
       mbar_init(bar(C::kBarQFull), 1);
       for (int s = 0; s < C::kStages; ++s) {
         mbar_init(bar(C::kBarKFull + s), 1);
-        mbar_init(bar(C::kBarKEmpty + s), 1);
         mbar_init(bar(C::kBarVFull + s), 1);
-        mbar_init(bar(C::kBarVEmpty + s), 1);
+        mbar_init(bar(C::kBarKVEmpty + s), 1);
       }
-      for (int b2 = 0; b2 < 2; ++b2) {
-        mbar_init(bar(C::kBarSFull + b2), 1);
-        mbar_init(bar(C::kBarSFree + b2), C::kSoftmaxThreads);
-        mbar_init(bar(C::kBarPFull + b2), C::kSoftmaxThreads);
+      for (int t = 0; t < 2; ++t) {
+        mbar_init(bar(C::kBarSFull + t), 1);
+        mbar_init(bar(C::kBarSFree + t), 4);  // one arrival per softmax warp of the tile
+        mbar_init(bar(C::kBarPFull + t), 4);
+        mbar_init(bar(C::kBarPVDone + t), 1);
+        mbar_init(bar(C::kBarOFinal + t), 1);
       }
-      mbar_init(bar(C::kBarPVDone), 1);
-      mbar_init(bar(C::kBarOFinal), 1);
+      mbar_init(bar(C::kBarDrain), 1);
       fence_mbar_init();
       tma_prefetch_desc(&p.tm_q);
       tma_prefetch_desc(&p.tm_k);
       tma_prefetch_desc(&p.tm_v);
     }
-  } else if (warp == 1) {
+  } else if (warp == C::kWarpMma) {
     tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
     tmem_relinquish();
-  } else if (warp == 2) {
-    // the ones matrix (E4M3 1.0 = 0x38) used to accumulate the row sums of P8
-    uint32_t* ones = reinterpret_cast<uint32_t*>(smem + C::kOnesOff);
-    for (int i = lane; i < 512; i += 32) ones[i] = 0x38383838u;
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int n = *count_slot;
+  const int n0 = count_slot[0], n1 = count_slot[1];
+  const int n_max = max(n0, n1);
 
-  if (warp == 0) {
+  if (warp == C::kWarpProducer) {
     // ---------------------------------------------------------------- producer
-    if (lane == 0 && n > 0) {
+    if (lane == 0 && n_max > 0) {
       const uint64_t pol_q = l2_policy_evict_first();
       const uint64_t pol_kv = l2_policy_evict_last();
-      mbar_arrive_expect_tx(bar(C::kBarQFull), C::kTileBytes);
-      tma_load_4d(base + C::kQOff, &p.tm_q, bar(C::kBarQFull), 0, qb * kTile, h, b, pol_q);
-      for (int it = 0; it < n; ++it) {
-        const int s = it % C::kStages;
-        const uint32_t ph = (it / C::kStages) & 1;
-        const int kv_row = static_cast<int>(list[it]) * kTile;
-        if (it >= C::kStages && !mbar_wait(bar(C::kBarKEmpty + s), ph ^ 1, abort_flag)) break;
-        mbar_arrive_expect_tx(bar(C::kBarKFull + s), C::kTileBytes);
-        tma_load_4d(base + C::kKOff + s * C::kTileBytes, &p.tm_k, bar(C::kBarKFull + s), 0, kv_row, g, b, pol_kv);
-        if (it >= C::kStages && !mbar_wait(bar(C::kBarVEmpty + s), ph ^ 1, abort_flag)) break;
-        mbar_arrive_expect_tx(bar(C::kBarVFull + s), C::kTileBytes);
-        tma_load_4d(base + C::kVOff + s * C::kTileBytes, &p.tm_v, bar(C::kBarVFull + s), 0, kv_row, g, b, pol_kv);
+      mbar_arrive_expect_tx(bar(C::kBarQFull), C::kTileBytes * ((n0 > 0) + (n1 > 0)));
+      if (n0 > 0) tma_load_4d(base + C::kQOff, &p.tm_q, bar(C::kBarQFull), 0, (2 * pr) * kTile, h, b, pol_q);
+      if (n1 > 0)
+        tma_load_4d(base + C::kQOff + C::kTileBytes, &p.tm_q, bar(C::kBarQFull), 0, (2 * pr + 1) * kTile, h, b,
+                    pol_q);
+      int seq = 0;
+      bool ok = true;
+      for (int j = 0; ok && j < n_max; ++j) {
+        for (int t = 0; t < 2; ++t) {
+          if (j >= (t ? n1 : n0)) continue;
+          const int s = seq % C::kStages;
+          const uint32_t round = static_cast<uint32_t>(seq / C::kStages);
+          if (seq >= C::kStages && !mbar_wait(bar(C::kBarKVEmpty + s), (round & 1) ^ 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const int kv_row = static_cast<int>(lists[t * kQbsaMaxKBlocks + j]) * kTile;
+          mbar_arrive_expect_tx(bar(C::kBarKFull + s), C::kTileBytes);
+          tma_load_4d(base + C::kKOff + s * C::kTileBytes, &p.tm_k, bar(C::kBarKFull + s), 0, kv_row, g, b, pol_kv);
+          mbar_arrive_expect_tx(bar(C::kBarVFull + s), C::kTileBytes);
+          tma_load_4d(base + C::kVOff + s * C::kTileBytes, &p.tm_v, bar(C::kBarVFull + s), 0, kv_row, g, b, pol_kv);
+          ++seq;
+        }
       }
+      // let the copies still in flight land before the CTA can exit (matters only after an abort)
+      for (int q = max(0, seq - C::kStages); q < seq; ++q) {
+        const uint32_t par = static_cast<uint32_t>(q / C::kStages) & 1;
+        mbar_wait_drain(bar(C::kBarKFull + q % C::kStages), par);
+        mbar_wait_drain(bar(C::kBarVFull + q % C::kStages), par);
+      }
+      mbar_wait_drain(bar(C::kBarQFull), 0);
     }
-  } else if (warp == 1) {
+  } else if (warp == C::kWarpMma) {
     // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0 && n > 0) {
+    if (lane == 0 && n_max > 0) {
       constexpr uint32_t idesc_qk = idesc_s8(128, 128);
       constexpr uint32_t idesc_pv = idesc_e4m3(128, 128, true);
       constexpr uint32_t idesc_pl = idesc_e4m3(128, 16, false);
       const uint32_t ones = base + C::kOnesOff;
       bool ok = mbar_wait(bar(C::kBarQFull), 0, abort_flag);
-      auto issue_pv = [&](int j) -> bool {
-        const int bj = j & 1;
-        const int s = j % C::kStages;
-        if (!mbar_wait(bar(C::kBarPFull + bj), (j >> 1) & 1, abort_flag)) return false;
-        if (!mbar_wait(bar(C::kBarVFull + s), (j / C::kStages) & 1, abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t vbase = base + C::kVOff + s * C::kTileBytes;
-        const uint32_t pcol = bj ? C::kColP1 : C::kColP0;
+      int seq = 0;
+      int last_seq[2] = {0, 0};     // ring sequence number of each tile's latest QK
+      int prev_t = -1, prev_j = 0;  // consumer of the S buffer's current contents
+      for (int j = 0; ok && j <= n_max; ++j) {
+        for (int t = 0; ok && t < 2; ++t) {
+          const int nt = t ? n1 : n0;
+          const int pv_seq = last_seq[t];  // stage of block j - 1 of this tile
+          if (j < nt) {
+            // S = Q_t K_jᵀ into the shared S buffer once its previous reader is done with it
+            const int s = seq % C::kStages;
+            if (!mbar_wait(bar(C::kBarKFull + s), static_cast<uint32_t>(seq / C::kStages) & 1, abort_flag)) {
+              ok = false;
+              break;
+            }
+            if (prev_t >= 0 &&
+                !mbar_wait(bar(C::kBarSFree + prev_t), static_cast<uint32_t>(prev_j) & 1, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t qbase = base + C::kQOff + t * C::kTileBytes;
+            const uint32_t kbase = base + C::kKOff + s * C::kTileBytes;
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          // 32 key rows per step: 8 TMEM columns of packed P8, 4096 B of V8
-          const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
-          mma_f8_ts(tmem + C::kColO, tmem + pcol + kk * 8, sdesc_sw128(vbase + kk * 4096, C::kTileBytes, 1024),
-                    idesc_pv, acc);
-          mma_f8_ts(tmem + C::kColL, tmem + pcol + kk * 8, sdesc_sw128(ones + kk * 32, 16, 1024), idesc_pl, acc);
-        }
-        mma_commit(bar(C::kBarPVDone));
-        mma_commit(bar(C::kBarVEmpty + s));
-        return true;
-      };
-      const uint32_t qbase = base + C::kQOff;
-      for (int it = 0; ok && it < n; ++it) {
-        const int s = it % C::kStages;
-        const int bi = it & 1;
-        if (!mbar_wait(bar(C::kBarKFull + s), (it / C::kStages) & 1, abort_flag)) { ok = false; break; }
-        if (it >= 2 && !mbar_wait(bar(C::kBarSFree + bi), ((it - 2) >> 1) & 1, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t kbase = base + C::kKOff + s * C::kTileBytes;
-        const uint32_t scol = bi ? C::kColS1 : C::kColS0;
+            for (int kk = 0; kk < 4; ++kk) {
+              mma_i8_ss(tmem + C::kColS, sdesc_sw128(qbase + kk * 32, 16, 1024),
+                        sdesc_sw128(kbase + kk * 32, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+            }
+            mma_commit(bar(C::kBarSFull + t));
+            prev_t = t;
+            prev_j = j;
+            last_seq[t] = seq;
+            ++seq;
+          }
+          if (j >= 1 && j - 1 < nt) {
+            // O_t += P_t V_{j-1}, L_t += P_t 1
+            const int s = pv_seq % C::kStages;
+            if (!mbar_wait(bar(C::kBarPFull + t), static_cast<uint32_t>(j - 1) & 1, abort_flag) ||
+                !mbar_wait(bar(C::kBarVFull + s), static_cast<uint32_t>(pv_seq / C::kStages) & 1, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t vbase = base + C::kVOff + s * C::kTileBytes;
+            const uint32_t pcol = tmem + C::kColP + 32 * t;
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          mma_i8_ss(tmem + scol, sdesc_sw128(qbase + kk * 32, 16, 1024), sdesc_sw128(kbase + kk * 32, 16, 1024),
-                    idesc_qk, kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk) {
+              // 32 key rows per step: 8 TMEM columns of packed P8, 4096 B of V8
+              const uint32_t acc = (j > 1 || kk > 0) ? 1u : 0u;
+              mma_f8_ts(tmem + C::kColO + 128 * t, pcol + kk * 8,
+                        sdesc_sw128(vbase + kk * 4096, C::kTileBytes, 1024), idesc_pv, acc);
+              mma_f8_ts(tmem + C::kColL + 16 * t, pcol + kk * 8, sdesc_sw128(ones + kk * 32, 16, 1024), idesc_pl,
+                        acc);
+            }
+            mma_commit(bar(C::kBarPVDone + t));
+            mma_commit(bar(C::kBarKVEmpty + s));
+            if (j == nt) mma_commit(bar(C::kBarOFinal + t));
+          }
         }
-        mma_commit(bar(C::kBarSFull + bi));
-        mma_commit(bar(C::kBarKEmpty + s));
-        if (it >= 1 && !issue_pv(it - 1)) { ok = false; break; }
       }
-      if (ok && issue_pv(n - 1)) mma_commit(bar(C::kBarOFinal));
+      // every MMA issued above has retired before TMEM can be released
+      mma_commit(bar(C::kBarDrain));
+      mbar_wait_drain(bar(C::kBarDrain), 0);
     }
   } else {
     // ---------------------------------------------------------------- softmax warps
+    const int t = warp >> 2;
     const int quarter = warp & 3;
-    const int half = (warp - 2) >> 2;  // 0: key columns [0,64), 1: [64,128)
     const int row = quarter * 32 + lane;
+    const int nt = t ? n1 : n0;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const int64_t i_glob = (int64_t)qb * kTile + row;
+    const int64_t i_glob = (int64_t)(2 * pr + t) * kTile + row;
     const float kNegInf = -__int_as_float(0x7f800000);
-    const uint32_t o_col = tmem + lane_off + C::kColO + half * 64;
-    const uint32_t l_col = tmem + lane_off + C::kColL;
+    const uint32_t s_col = tmem + lane_off + C::kColS;
+    const uint32_t o_col = tmem + lane_off + C::kColO + 128 * t;
+    const uint32_t l_col = tmem + lane_off + C::kColL + 16 * t;
+    const uint32_t p_col = tmem + lane_off + C::kColP + 32 * t;
+    const uint16_t* list = lists + t * kQbsaMaxKBlocks;
+    const float* cst_list = csts + t * kQbsaMaxKBlocks;
 
     float m = kNegInf;    // running max, log2 domain
     float ref = kNegInf;  // power-of-two reference of the FP8 weights (an integer)
     bool ok = true;
-    for (int it = 0; it < n; ++it) {
-      const int kb = list[it];
-      const int bi = it & 1;
-      const float cst = cst_list[it];
-      const int valid = min(kTile, p.Skv - kb * kTile) - half * 64;  // valid columns of this half
-      // never leave the loop early (the paired warp waits on named barriers below)
-      if (ok) ok = mbar_wait(bar(C::kBarSFull + bi), (it >> 1) & 1, abort_flag);
+    for (int j = 0; ok && j < nt; ++j) {
+      const int kb = list[j];
+      const float cst = cst_list[j];
+      const int valid = min(kTile, p.Skv - kb * kTile);  // key columns inside S_kv
+      ok = warp_wait(bar(C::kBarSFull + t), static_cast<uint32_t>(j) & 1, abort_flag);
+      if (!ok) break;
       tc_fence_after();
-      float sv[64];  // exact: |dot| <= 128 * 127^2 < 2^24
+      float sv[128];  // exact: |dot| <= 128 * 127^2 < 2^24
       {
-        uint32_t r[64];
-        tmem_ld64_wait(tmem + lane_off + (bi ? C::kColS1 : C::kColS0) + half * 64, r);
+        uint32_t rr[128];
+        tmem_ld128_wait(s_col, rr);
 #pragma unroll
-        for (int x = 0; x < 64; ++x) sv[x] = __int2float_rn(static_cast<int32_t>(r[x]));
+        for (int x = 0; x < 128; ++x) sv[x] = __int2float_rn(static_cast<int32_t>(rr[x]));
       }
       tc_fence_before();
-      mbar_arrive(bar(C::kBarSFree + bi));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(C::kBarSFree + t));
 
-      if (valid < 64) {  // tail block: keys past S_kv get -inf (p = 0 below)
+      // row max of z = t * c: max(t) * c for c >= 0, min(t) * c otherwise (c is uniform)
+      const bool pos = cst >= 0.f;
+      if (valid < kTile) {  // tail block: keys past S_kv take no part
+        const float pad = pos ? kNegInf : -kNegInf;
 #pragma unroll
-        for (int x = 0; x < 64; ++x)
-          if (x >= valid) sv[x] = kNegInf;
+        for (int x = 0; x < 128; ++x)
+          if (x >= valid) sv[x] = pad;
       }
-      const float pmax = max64(sv);
-      float* slot = xch + (it & 1) * 256;
-      slot[half * 128 + row] = pmax;
-      qbsa_named_bar_sync(1 + quarter, 64);
-      const float tmax = fmaxf(pmax, slot[(half ^ 1) * 128 + row]);
-
-      // max(t) * c == max(t * c): multiplication by c > 0 is monotone in float
-      const float m_blk = tmax * cst;
+      const float m_blk = (pos ? max128(sv) : min128(sv)) * cst;
       m = fmaxf(m, m_blk);
       // power-of-two reference: re-set to ceil(m) once m exceeds it by more than 8, so
       // p <= 2^8 stays below E4M3's 448 and every rescale is an exact power of two
@@ -299,55 +363,67 @@ __global__ void __launch_bounds__(320, 1) attn_qbsa_kernel(const __grid_constant
       const int dexp = need ? static_cast<int>(ref - new_ref) : 0;
       const float a = (dexp < -126) ? 0.f : __int_as_float((127 + dexp) << 23);
       ref = new_ref;
-      if (__any_sync(0xffffffffu, need)) {
-        if (ok) ok = mbar_wait(bar(C::kBarPVDone), (it - 1) & 1, abort_flag);
-        tc_fence_after();
-        uint32_t r[32];
-#pragma unroll
-        for (int ch = 0; ch < 2; ++ch) {
-          tmem_ld32_wait(o_col + ch * 32, r);
-#pragma unroll
-          for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(__uint_as_float(r[x]) * a);
-          tmem_st32(o_col + ch * 32, r);
-        }
-        if (half == 0) tmem_st1(l_col, __float_as_uint(__uint_as_float(tmem_ld1_wait(l_col)) * a));
-        tmem_st_wait();
-      }
+
       // p = 2^(t c - R) held in FP16 (the precision of P before its FP8 rounding),
-      // two weights per ex2, then rounded to E4M3
-      uint32_t pk[16];
+      // then rounded to E4M3; four weights per packed word
+      const uint64_t cc = pack_f32x2(cst, cst);
+      const uint64_t nr = pack_f32x2(-ref, -ref);
+      uint32_t pk[32];
 #pragma unroll
-      for (int x = 0; x < 16; ++x) {
-        pk[x] = exp2_e4m3x4(fmaf(sv[4 * x], cst, -ref), fmaf(sv[4 * x + 1], cst, -ref),
-                            fmaf(sv[4 * x + 2], cst, -ref), fmaf(sv[4 * x + 3], cst, -ref));
+      for (int x = 0; x < 32; ++x)
+        pk[x] = fma_exp2_e4m3x4(sv[4 * x], sv[4 * x + 1], sv[4 * x + 2], sv[4 * x + 3], cc, nr);
+      if (valid < kTile) {  // tail block: zero the weights of keys past S_kv whatever c is
+#pragma unroll
+        for (int x = 0; x < 32; ++x) {
+          const int keep = min(max(valid - 4 * x, 0), 4);
+          pk[x] &= (keep == 4) ? 0xffffffffu : ((1u << (8 * keep)) - 1u);
+        }
       }
-      tmem_st16(tmem + lane_off + (bi ? C::kColP1 : C::kColP0) + half * 16, pk);
+
+      // P_t and O_t are free once the previous block's P·V has retired
+      if (j > 0) {
+        ok = warp_wait(bar(C::kBarPVDone + t), static_cast<uint32_t>(j - 1) & 1, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, need)) {
+          uint32_t rr[32];
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch) {
+            tmem_ld32_wait(o_col + ch * 32, rr);
+#pragma unroll
+            for (int x = 0; x < 32; ++x) rr[x] = __float_as_uint(__uint_as_float(rr[x]) * a);
+            tmem_st32(o_col + ch * 32, rr);
+          }
+          tmem_st1(l_col, __float_as_uint(__uint_as_float(tmem_ld1_wait(l_col)) * a));
+        }
+      }
+      tmem_st32(p_col, pk);
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(bar(C::kBarPFull + bi));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(C::kBarPFull + t));
     }
 
     // ------------------------------------------------------------ epilogue
     const bool row_valid = i_glob < p.Sq;
-    bool have_o = ok && n > 0;
+    bool have_o = ok && nt > 0;
     if (have_o) {
       // a dedicated single-use barrier: pv_done's parity cannot tell PV(n-1) from PV(n-3)
-      have_o = mbar_wait(bar(C::kBarOFinal), 0, abort_flag);
+      have_o = warp_wait(bar(C::kBarOFinal + t), 0, abort_flag);
       tc_fence_after();
     }
     float l = 0.f;
     if (have_o) l = __uint_as_float(tmem_ld1_wait(l_col));
     const float inv_l = (l > 0.f) ? 1.0f / l : 0.f;
-    const float* vsc = p.v_scale + ((int64_t)b * p.Nkv + g) * 128 + half * 64;
-    __nv_bfloat16* orow = p.out + (((int64_t)b * p.Nq + h) * p.Sq + i_glob) * 128 + half * 64;
+    __nv_bfloat16* orow = p.out + (((int64_t)b * p.Nq + h) * p.Sq + i_glob) * 128;
 #pragma unroll
-    for (int ch = 0; ch < 2; ++ch) {
-      uint32_t r[32];
+    for (int ch = 0; ch < 4; ++ch) {
+      uint32_t rr[32];
       if (have_o) {
-        tmem_ld32_wait(o_col + ch * 32, r);
+        tmem_ld32_wait(o_col + ch * 32, rr);
       } else {
 #pragma unroll
-        for (int x = 0; x < 32; ++x) r[x] = 0u;
+        for (int x = 0; x < 32; ++x) rr[x] = 0u;
       }
       if (row_valid) {
         uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
@@ -355,7 +431,7 @@ __global__ void __launch_bounds__(320, 1) attn_qbsa_kernel(const __grid_constant
         for (int x = 0; x < 4; ++x) {
           float f[8];
 #pragma unroll
-          for (int y = 0; y < 8; ++y) f[y] = __uint_as_float(r[8 * x + y]) * (vsc[ch * 32 + 8 * x + y] * inv_l);
+          for (int y = 0; y < 8; ++y) f[y] = __uint_as_float(rr[8 * x + y]) * (vsc[ch * 32 + 8 * x + y] * inv_l);
           uint4 v;
           v.x = pack_bf16x2(f[0], f[1]);
           v.y = pack_bf16x2(f[2], f[3]);
@@ -365,7 +441,7 @@ __global__ void __launch_bounds__(320, 1) attn_qbsa_kernel(const __grid_constant
         }
       }
     }
-    if (half == 0 && row_valid) {
+    if (row_valid) {
       const int64_t sidx = ((int64_t)b * p.Nq + h) * p.Sq + i_glob;
       const bool live = l > 0.f;
       if (p.softmax_max) p.softmax_max[sidx] = live ? m * 0.6931471805599453f : kNegInf;
@@ -375,7 +451,7 @@ __global__ void __launch_bounds__(320, 1) attn_qbsa_kernel(const __grid_constant
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == C::kWarpMma) {
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmemCols);
   }

@@ -84,6 +84,20 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   }
 }
 
+// Cleanup wait: bounded by the same time limit but not by the abort flag, so a CTA that
+// aborted can still let its own asynchronous copies and MMAs land before it exits.
+__device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 0 && global_timer_ns() - t0 > QBSA_WAIT_TIMEOUT_NS) {
+      atomicCAS(&g_device_error, 0u, static_cast<unsigned int>(kErrTimeout));
+      return false;
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------------
 // TMA (no multicast anywhere in this library)
 // ---------------------------------------------------------------------------------
@@ -396,6 +410,74 @@ __device__ __forceinline__ uint32_t exp2_e4m3x4(float x0, float x1, float x2, fl
       : "=r"(r)
       : "f"(x0), "f"(x1), "f"(x2), "f"(x3));
   return r;
+}
+
+// Two f32 in one 64-bit register pair (lo = element 0), for the packed f32x2 ops.
+__device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+
+// Four scores s (exact integers held in f32) -> z = s * c - R with two packed
+// fma.rn.f32x2 (cc = {c, c}, nr = {-R, -R}) -> 2^z (fp32 ex2) rounded to FP16 -> four
+// E4M3 bytes (byte i = value i); both roundings nearest even, the second saturating.
+__device__ __forceinline__ uint32_t fma_exp2_e4m3x4(float s0, float s1, float s2, float s3, uint64_t cc,
+                                                    uint64_t nr) {
+  uint32_t r;
+  asm("{\n\t.reg .f32 e0, e1, e2, e3;\n\t.reg .b64 a01, a23, z01, z23;\n\t.reg .b32 h01, h23;\n\t"
+      ".reg .b16 lo, hi;\n\t"
+      "mov.b64 a01, {%1, %2};\n\t"
+      "mov.b64 a23, {%3, %4};\n\t"
+      "fma.rn.f32x2 z01, a01, %5, %6;\n\t"
+      "fma.rn.f32x2 z23, a23, %5, %6;\n\t"
+      "mov.b64 {e0, e1}, z01;\n\t"
+      "mov.b64 {e2, e3}, z23;\n\t"
+      "ex2.approx.ftz.f32 e0, e0;\n\t"
+      "ex2.approx.ftz.f32 e1, e1;\n\t"
+      "ex2.approx.ftz.f32 e2, e2;\n\t"
+      "ex2.approx.ftz.f32 e3, e3;\n\t"
+      "cvt.rn.f16x2.f32 h01, e1, e0;\n\t"
+      "cvt.rn.f16x2.f32 h23, e3, e2;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f16x2 lo, h01;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f16x2 hi, h23;\n\t"
+      "mov.b32 %0, {lo, hi};\n\t}"
+      : "=r"(r)
+      : "f"(s0), "f"(s1), "f"(s2), "f"(s3), "l"(cc), "l"(nr));
+  return r;
+}
+
+// Three-input minimum (one instruction on sm_100).
+__device__ __forceinline__ float fmin3(float a, float b, float c) {
+  float d;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Maximum / minimum of 128 values as trees of three-input ops (64 instructions).
+__device__ __forceinline__ float max128(const float (&v)[128]) {
+  float a[43], b[15], c[5];
+#pragma unroll
+  for (int i = 0; i < 42; ++i) a[i] = fmax3(v[3 * i], v[3 * i + 1], v[3 * i + 2]);
+  a[42] = fmaxf(v[126], v[127]);
+#pragma unroll
+  for (int i = 0; i < 14; ++i) b[i] = fmax3(a[3 * i], a[3 * i + 1], a[3 * i + 2]);
+  b[14] = a[42];
+#pragma unroll
+  for (int i = 0; i < 5; ++i) c[i] = fmax3(b[3 * i], b[3 * i + 1], b[3 * i + 2]);
+  return fmax3(fmax3(c[0], c[1], c[2]), c[3], c[4]);
+}
+__device__ __forceinline__ float min128(const float (&v)[128]) {
+  float a[43], b[15], c[5];
+#pragma unroll
+  for (int i = 0; i < 42; ++i) a[i] = fmin3(v[3 * i], v[3 * i + 1], v[3 * i + 2]);
+  a[42] = fminf(v[126], v[127]);
+#pragma unroll
+  for (int i = 0; i < 14; ++i) b[i] = fmin3(a[3 * i], a[3 * i + 1], a[3 * i + 2]);
+  b[14] = a[42];
+#pragma unroll
+  for (int i = 0; i < 5; ++i) c[i] = fmin3(b[3 * i], b[3 * i + 1], b[3 * i + 2]);
+  return fmin3(fmin3(c[0], c[1], c[2]), c[3], c[4]);
 }
 
 }  // namespace qbsa

@@ -357,10 +357,11 @@ qbsa_status qbsa_fwd(const int8_t* q_i8, const int8_t* k_i8, const float* q_bloc
   prm.nqb = nqb;
   prm.nkb = nkb;
   prm.scale_log2 = scale * 1.4426950408889634f;
-  prm.n_rank = B * nqb;
+  prm.n_pair = (nqb + 1) / 2;
+  prm.n_rank = B * prm.n_pair;
   // K8 + V8 bytes of one query head: one kv head over all batches, shared by the group
   prm.head_grp = head_group(static_cast<double>(std::max(Skv, 1)) * 128 * 2 * B / prm.group, Nq);
-  const int64_t n_work = (int64_t)B * nqb * Nq;
+  const int64_t n_work = (int64_t)B * prm.n_pair * Nq;
   if (n_work > 0x7fffffffLL) return fail(QBSA_ERR_UNSUPPORTED, "too many query blocks");
   if (Skv == 0) {
     // no key: every row is fully masked; keep the kernel path (no block is visited)

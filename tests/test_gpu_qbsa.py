@@ -6,7 +6,7 @@ import torch
 
 import quantized_block_sparse_attn_b200 as qb
 from oracle import dense, quant
-from workloads import CONFIGS, block_keep_mask, blocky_qk_bf16, iid_normal_bf16, sample_rows
+from workloads import CONFIGS, block_keep_mask, blocky_qk_bf16, iid_normal_bf16, random_atten_mask, sample_rows
 from tests.gpu_util import QUANT_MAX_ABS, compare_out, compare_stats, dev, dev_bf16, host_f64
 
 pytestmark = pytest.mark.gpu
@@ -39,6 +39,32 @@ def test_qbsa_parity_small(B, Nq, Nkv, Sq, Skv, keep):
     q8, qs, k8, ks, v8, vs = _quantized(q, k, v)
     bm = block_keep_mask(20, B, Nq, -(-Sq // 128), -(-Skv // 128), keep)
     scale = D ** -0.5
+    got, gmax, gsum = _run(q8, qs, k8, ks, v8, vs, bm, scale)
+    ref, rmax, rsum = quant.qbsa_forward(q8, k8, qs, ks, v8, vs, bm, scale)
+    compare_out(got, ref, QUANT_MAX_ABS)
+    compare_stats(gmax, gsum, rmax, rsum)
+
+
+@pytest.mark.parametrize("sign", [1.0, -1.0])
+def test_qbsa_unequal_tile_pairs(sign):
+    """Query blocks are processed in pairs: unequal kept counts, one side empty, an odd
+    last pair, a ragged key tail; a negative scale exercises the row-minimum path."""
+    B, Nq, Nkv, Sq, Skv, D = 1, 2, 1, 640, 700, 128
+    nqb, nkb = 5, 6
+    q = iid_normal_bf16(23, 0, B, Nq, Sq, D)
+    k = iid_normal_bf16(23, 1, B, Nkv, Skv, D)
+    v = iid_normal_bf16(23, 2, B, Nkv, Skv, D)
+    q8, qs, k8, ks, v8, vs = _quantized(q, k, v)
+    bm = (random_atten_mask(23, (B, Nq, nqb, nkb), 0.5) == 0).astype(np.uint8)
+    bm[0, 0, 0, :] = 0          # pair 0 of head 0: first tile empty, second not
+    bm[0, 0, 1, :] = 1
+    bm[0, 0, 3, :] = 0          # pair 1 of head 0: second tile empty
+    bm[0, 0, 2, :] = 0
+    bm[0, 0, 2, 5] = 1          # ... first tile keeps only the ragged tail block
+    bm[0, 1, 0, :] = 0
+    bm[0, 1, 0, 2] = 1          # head 1, pair 0: 1 block against a full row
+    bm[0, 1, 1, :] = 1
+    scale = sign * D ** -0.5
     got, gmax, gsum = _run(q8, qs, k8, ks, v8, vs, bm, scale)
     ref, rmax, rsum = quant.qbsa_forward(q8, k8, qs, ks, v8, vs, bm, scale)
     compare_out(got, ref, QUANT_MAX_ABS)
