@@ -22,12 +22,13 @@
 //               O * v_scale / L -> bf16.
 //   warp 8      TMA producer: Q of both tiles once; K and V tiles of the kept blocks
 //               of both tiles, interleaved (t0 j, t1 j, t0 j+1, ...), 5-stage ring.
-//   warp 9      TMEM owner + MMA issuer, in the order QK0(j), PV0(j-1), QK1(j),
-//               PV1(j-1): S = Q8 K8ᵀ (kind::i8, s32 into the one shared S buffer),
-//               O_t += P8_t V8 (kind::f8f6f4, A = P8 from TMEM, B = V8 MN-major) and
-//               L_t += P8_t · 1 (N = 16 ones matrix), so L is exactly Σ p8.
-// TMEM columns: O0 [0,128) O1 [128,256) S [256,384) P0 [384,416) P1 [416,448)
-//               L0 [448,464) L1 [464,480).
+//   warp 9      TMEM owner + QK issuer: S = Q8_t K8ᵀ (kind::i8, s32 into the one
+//               shared S buffer) once the S buffer's previous reader is done.
+//   warp 10     PV issuer: [O_t | L_t] += P8_t [V8 | 1] as one N = 144 MMA
+//               (kind::f8f6f4, A = P8 from TMEM, B MN-major: V8's 128 channels plus a
+//               16-column ones block in shared memory), so L is exactly Σ p8.
+// The two issuers block independently while the tensor core drains their queues.
+// TMEM columns: O0|L0 [0,144) S [160,288) O1|L1 [288,432) P0 [448,480) P1 [480,512).
 //
 // CTA order: query heads in groups whose K8/V8 fit in about 48 MB of L2, query-block
 // pairs in order, heads fastest inside a group.
@@ -68,28 +69,28 @@ struct QbsaCfg {
   static constexpr int kQOff = 0;                   // Q of tile 0, then tile 1
   static constexpr int kKOff = kQOff + 2 * kTileBytes;
   static constexpr int kVOff = kKOff + kStages * kTileBytes;
-  static constexpr int kOnesOff = kVOff + kStages * kTileBytes;   // 16 x 128 bytes of E4M3 1.0
-  static constexpr int kCOff = kOnesOff + 2048;                    // float [2][kMax] dequant constants
+  static constexpr int kOnesOff = kVOff + kStages * kTileBytes;   // 32 rows x 128 B of E4M3 1.0
+  static constexpr int kCOff = kOnesOff + 4096;                    // float [2][kMax] dequant constants
   static constexpr int kListOff = kCOff + 2 * kQbsaMaxKBlocks * 4;  // uint16 [2][kMax] kept blocks
   static constexpr int kVscOff = kListOff + 2 * kQbsaMaxKBlocks * 2;  // float [128] value scales
   static constexpr int kBarOff = kVscOff + 128 * 4;
   static constexpr int kBarQFull = 0;
-  static constexpr int kBarKFull = 1;
-  static constexpr int kBarVFull = kBarKFull + kStages;
-  static constexpr int kBarKVEmpty = kBarVFull + kStages;
+  static constexpr int kBarKVFull = 1;
+  static constexpr int kBarKVEmpty = kBarKVFull + kStages;
   static constexpr int kBarSFull = kBarKVEmpty + kStages;  // [2], per tile
   static constexpr int kBarSFree = kBarSFull + 2;          // [2], per tile
   static constexpr int kBarPFull = kBarSFree + 2;          // [2]
   static constexpr int kBarPVDone = kBarPFull + 2;         // [2]
   static constexpr int kBarOFinal = kBarPVDone + 2;        // [2], single use
-  static constexpr int kBarDrain = kBarOFinal + 2;         // single use: every MMA retired
-  static constexpr int kNumBars = kBarDrain + 1;
+  static constexpr int kBarDrain = kBarOFinal + 2;         // [2] single use: every MMA of an issuer retired
+  static constexpr int kNumBars = kBarDrain + 2;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // tmem addr, abort flag, counts[2]
   static constexpr int kSmemBytes = kMiscOff + 16 + 1024;
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr uint32_t kColO = 0, kColS = 256, kColP = 384, kColL = 448;  // O_t = kColO + 128 t, ...
-  static constexpr int kThreads = 320;
-  static constexpr int kWarpProducer = 8, kWarpMma = 9;
+  // O_t|L_t at kColO[t] (L_t = its column 128), P_t at kColP + 32 t
+  static constexpr uint32_t kColO0 = 0, kColS = 160, kColO1 = 288, kColP = 448;
+  static constexpr int kThreads = 352;
+  static constexpr int kWarpProducer = 8, kWarpQK = 9, kWarpPV = 10;
 };
 static_assert(QbsaCfg::kSmemBytes <= 232448, "shared memory above the 227 KB opt-in limit");
 
@@ -107,12 +108,16 @@ __device__ __forceinline__ int compact_mask_row(const uint8_t* row, int n_kb, ui
   return count;
 }
 
-// Every lane waits; the warp proceeds only if all lanes saw the phase complete.
+// Lane 0 waits for the phase; the warp synchronises on it (callers then fence with
+// tcgen05.fence::after_thread_sync before touching TMEM).
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
-  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag)) != 0;
+  int ok = 1;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort_flag) ? 1 : 0;
+  __syncwarp();
+  return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
-__global__ void __launch_bounds__(320, 1) attn_qbsa_kernel(const __grid_constant__ QbsaParams p) {
+__global__ void __launch_bounds__(352, 1) attn_qbsa_kernel(const __grid_constant__ QbsaParams p) {
   using C = QbsaCfg;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
@@ -159,9 +164,9 @@ __global__ void __launch_bounds__(320, 1) attn_qbsa_kernel(const __grid_constant
     }
     if (lane == 0) count_slot[t] = cnt;
   } else if (warp == 1) {
-    // the ones matrix (E4M3 1.0 = 0x38) used to accumulate the row sums of P8
+    // the ones block (E4M3 1.0 = 0x38) that turns the P·V MMA's columns 128..143 into Σ p8
     uint32_t* ones = reinterpret_cast<uint32_t*>(smem + C::kOnesOff);
-    for (int i = lane; i < 512; i += 32) ones[i] = 0x38383838u;
+    for (int i = lane; i < 1024; i += 32) ones[i] = 0x38383838u;
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   } else if (warp == 2) {
     const float* vs = p.v_scale + ((int64_t)b * p.Nkv + g) * 128;
@@ -171,8 +176,7 @@ __global__ void __launch_bounds__(320, 1) attn_qbsa_kernel(const __grid_constant
       *abort_flag = 0;
       mbar_init(bar(C::kBarQFull), 1);
       for (int s = 0; s < C::kStages; ++s) {
-        mbar_init(bar(C::kBarKFull + s), 1);
-        mbar_init(bar(C::kBarVFull + s), 1);
+        mbar_init(bar(C::kBarKVFull + s), 1);
         mbar_init(bar(C::kBarKVEmpty + s), 1);
       }
       for (int t = 0; t < 2; ++t) {
@@ -183,12 +187,13 @@ __global__ void __launch_bounds__(320, 1) attn_qbsa_kernel(const __grid_constant
         mbar_init(bar(C::kBarOFinal + t), 1);
       }
       mbar_init(bar(C::kBarDrain), 1);
+      mbar_init(bar(C::kBarDrain + 1), 1);
       fence_mbar_init();
       tma_prefetch_desc(&p.tm_q);
       tma_prefetch_desc(&p.tm_k);
       tma_prefetch_desc(&p.tm_v);
     }
-  } else if (warp == C::kWarpMma) {
+  } else if (warp == C::kWarpQK) {
     tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
     tmem_relinquish();
   }
@@ -221,91 +226,90 @@ __global__ void __launch_bounds__(320, 1) attn_qbsa_kernel(const __grid_constant
             break;
           }
           const int kv_row = static_cast<int>(lists[t * kQbsaMaxKBlocks + j]) * kTile;
-          mbar_arrive_expect_tx(bar(C::kBarKFull + s), C::kTileBytes);
-          tma_load_4d(base + C::kKOff + s * C::kTileBytes, &p.tm_k, bar(C::kBarKFull + s), 0, kv_row, g, b, pol_kv);
-          mbar_arrive_expect_tx(bar(C::kBarVFull + s), C::kTileBytes);
-          tma_load_4d(base + C::kVOff + s * C::kTileBytes, &p.tm_v, bar(C::kBarVFull + s), 0, kv_row, g, b, pol_kv);
+          mbar_arrive_expect_tx(bar(C::kBarKVFull + s), 2 * C::kTileBytes);
+          tma_load_4d(base + C::kKOff + s * C::kTileBytes, &p.tm_k, bar(C::kBarKVFull + s), 0, kv_row, g, b, pol_kv);
+          tma_load_4d(base + C::kVOff + s * C::kTileBytes, &p.tm_v, bar(C::kBarKVFull + s), 0, kv_row, g, b, pol_kv);
           ++seq;
         }
       }
       // let the copies still in flight land before the CTA can exit (matters only after an abort)
       for (int q = max(0, seq - C::kStages); q < seq; ++q) {
-        const uint32_t par = static_cast<uint32_t>(q / C::kStages) & 1;
-        mbar_wait_drain(bar(C::kBarKFull + q % C::kStages), par);
-        mbar_wait_drain(bar(C::kBarVFull + q % C::kStages), par);
+        mbar_wait_drain(bar(C::kBarKVFull + q % C::kStages), static_cast<uint32_t>(q / C::kStages) & 1);
       }
       mbar_wait_drain(bar(C::kBarQFull), 0);
     }
-  } else if (warp == C::kWarpMma) {
-    // ---------------------------------------------------------------- MMA issuer
+  } else if (warp == C::kWarpQK) {
+    // ---------------------------------------------------------------- QK issuer
     if (lane == 0 && n_max > 0) {
       constexpr uint32_t idesc_qk = idesc_s8(128, 128);
-      constexpr uint32_t idesc_pv = idesc_e4m3(128, 128, true);
-      constexpr uint32_t idesc_pl = idesc_e4m3(128, 16, false);
-      const uint32_t ones = base + C::kOnesOff;
       bool ok = mbar_wait(bar(C::kBarQFull), 0, abort_flag);
       int seq = 0;
-      int last_seq[2] = {0, 0};     // ring sequence number of each tile's latest QK
-      int prev_t = -1, prev_j = 0;  // consumer of the S buffer's current contents
-      for (int j = 0; ok && j <= n_max; ++j) {
+      int prev_t = -1, prev_j = 0;  // reader of the S buffer's current contents
+      for (int j = 0; ok && j < n_max; ++j) {
         for (int t = 0; ok && t < 2; ++t) {
-          const int nt = t ? n1 : n0;
-          const int pv_seq = last_seq[t];  // stage of block j - 1 of this tile
-          if (j < nt) {
-            // S = Q_t K_jᵀ into the shared S buffer once its previous reader is done with it
-            const int s = seq % C::kStages;
-            if (!mbar_wait(bar(C::kBarKFull + s), static_cast<uint32_t>(seq / C::kStages) & 1, abort_flag)) {
-              ok = false;
-              break;
-            }
-            if (prev_t >= 0 &&
-                !mbar_wait(bar(C::kBarSFree + prev_t), static_cast<uint32_t>(prev_j) & 1, abort_flag)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint32_t qbase = base + C::kQOff + t * C::kTileBytes;
-            const uint32_t kbase = base + C::kKOff + s * C::kTileBytes;
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              mma_i8_ss(tmem + C::kColS, sdesc_sw128(qbase + kk * 32, 16, 1024),
-                        sdesc_sw128(kbase + kk * 32, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
-            }
-            mma_commit(bar(C::kBarSFull + t));
-            prev_t = t;
-            prev_j = j;
-            last_seq[t] = seq;
-            ++seq;
+          if (j >= (t ? n1 : n0)) continue;
+          const int s = seq % C::kStages;
+          if (!mbar_wait(bar(C::kBarKVFull + s), static_cast<uint32_t>(seq / C::kStages) & 1, abort_flag) ||
+              (prev_t >= 0 &&
+               !mbar_wait(bar(C::kBarSFree + prev_t), static_cast<uint32_t>(prev_j) & 1, abort_flag))) {
+            ok = false;
+            break;
           }
-          if (j >= 1 && j - 1 < nt) {
-            // O_t += P_t V_{j-1}, L_t += P_t 1
-            const int s = pv_seq % C::kStages;
-            if (!mbar_wait(bar(C::kBarPFull + t), static_cast<uint32_t>(j - 1) & 1, abort_flag) ||
-                !mbar_wait(bar(C::kBarVFull + s), static_cast<uint32_t>(pv_seq / C::kStages) & 1, abort_flag)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint32_t vbase = base + C::kVOff + s * C::kTileBytes;
-            const uint32_t pcol = tmem + C::kColP + 32 * t;
+          tc_fence_after();
+          const uint32_t qbase = base + C::kQOff + t * C::kTileBytes;
+          const uint32_t kbase = base + C::kKOff + s * C::kTileBytes;
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              // 32 key rows per step: 8 TMEM columns of packed P8, 4096 B of V8
-              const uint32_t acc = (j > 1 || kk > 0) ? 1u : 0u;
-              mma_f8_ts(tmem + C::kColO + 128 * t, pcol + kk * 8,
-                        sdesc_sw128(vbase + kk * 4096, C::kTileBytes, 1024), idesc_pv, acc);
-              mma_f8_ts(tmem + C::kColL + 16 * t, pcol + kk * 8, sdesc_sw128(ones + kk * 32, 16, 1024), idesc_pl,
-                        acc);
-            }
-            mma_commit(bar(C::kBarPVDone + t));
-            mma_commit(bar(C::kBarKVEmpty + s));
-            if (j == nt) mma_commit(bar(C::kBarOFinal + t));
+          for (int kk = 0; kk < 4; ++kk) {
+            mma_i8_ss(tmem + C::kColS, sdesc_sw128(qbase + kk * 32, 16, 1024), sdesc_sw128(kbase + kk * 32, 16, 1024),
+                      idesc_qk, kk > 0 ? 1u : 0u);
           }
+          mma_commit(bar(C::kBarSFull + t));
+          prev_t = t;
+          prev_j = j;
+          ++seq;
         }
       }
       // every MMA issued above has retired before TMEM can be released
       mma_commit(bar(C::kBarDrain));
       mbar_wait_drain(bar(C::kBarDrain), 0);
+    }
+  } else if (warp == C::kWarpPV) {
+    // ---------------------------------------------------------------- PV issuer
+    if (lane == 0 && n_max > 0) {
+      constexpr uint32_t idesc_pv = idesc_e4m3(128, 144, true);
+      const uint32_t ones = base + C::kOnesOff;
+      bool ok = true;
+      int seq = 0;
+      for (int j = 0; ok && j < n_max; ++j) {
+        for (int t = 0; ok && t < 2; ++t) {
+          const int nt = t ? n1 : n0;
+          if (j >= nt) continue;
+          const int s = seq % C::kStages;
+          if (!mbar_wait(bar(C::kBarPFull + t), static_cast<uint32_t>(j) & 1, abort_flag) ||
+              !mbar_wait(bar(C::kBarKVFull + s), static_cast<uint32_t>(seq / C::kStages) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t vbase = base + C::kVOff + s * C::kTileBytes;
+          const uint32_t pcol = tmem + C::kColP + 32 * t;
+          const uint32_t ocol = tmem + (t ? C::kColO1 : C::kColO0);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            // 32 key rows per step: 8 TMEM columns of packed P8; B = 4096 B of V8 (MN atom 0)
+            // and, one leading-byte offset further, the same 32 rows of the ones block (atom 1)
+            const uint32_t vk = vbase + kk * 4096;
+            mma_f8_ts(ocol, pcol + kk * 8, sdesc_sw128(vk, ones - vk, 1024), idesc_pv,
+                      (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(bar(C::kBarPVDone + t));
+          mma_commit(bar(C::kBarKVEmpty + s));
+          if (j == nt - 1) mma_commit(bar(C::kBarOFinal + t));
+          ++seq;
+        }
+      }
+      mma_commit(bar(C::kBarDrain + 1));
+      mbar_wait_drain(bar(C::kBarDrain + 1), 0);
     }
   } else {
     // ---------------------------------------------------------------- softmax warps
@@ -317,8 +321,8 @@ __global__ void __launch_bounds__(320, 1) attn_qbsa_kernel(const __grid_constant
     const int64_t i_glob = (int64_t)(2 * pr + t) * kTile + row;
     const float kNegInf = -__int_as_float(0x7f800000);
     const uint32_t s_col = tmem + lane_off + C::kColS;
-    const uint32_t o_col = tmem + lane_off + C::kColO + 128 * t;
-    const uint32_t l_col = tmem + lane_off + C::kColL + 16 * t;
+    const uint32_t o_col = tmem + lane_off + (t ? C::kColO1 : C::kColO0);
+    const uint32_t l_col = o_col + 128;
     const uint32_t p_col = tmem + lane_off + C::kColP + 32 * t;
     const uint16_t* list = lists + t * kQbsaMaxKBlocks;
     const float* cst_list = csts + t * kQbsaMaxKBlocks;
@@ -333,13 +337,8 @@ __global__ void __launch_bounds__(320, 1) attn_qbsa_kernel(const __grid_constant
       ok = warp_wait(bar(C::kBarSFull + t), static_cast<uint32_t>(j) & 1, abort_flag);
       if (!ok) break;
       tc_fence_after();
-      float sv[128];  // exact: |dot| <= 128 * 127^2 < 2^24
-      {
-        uint32_t rr[128];
-        tmem_ld128_wait(s_col, rr);
-#pragma unroll
-        for (int x = 0; x < 128; ++x) sv[x] = __int2float_rn(static_cast<int32_t>(rr[x]));
-      }
+      uint32_t sv[128];  // s32 scores; exact in f32 since |dot| <= 128 * 127^2 < 2^24
+      tmem_ld128_wait(s_col, sv);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(C::kBarSFree + t));
@@ -347,12 +346,12 @@ __global__ void __launch_bounds__(320, 1) attn_qbsa_kernel(const __grid_constant
       // row max of z = t * c: max(t) * c for c >= 0, min(t) * c otherwise (c is uniform)
       const bool pos = cst >= 0.f;
       if (valid < kTile) {  // tail block: keys past S_kv take no part
-        const float pad = pos ? kNegInf : -kNegInf;
+        const uint32_t pad = pos ? 0x80000000u : 0x7fffffffu;
 #pragma unroll
         for (int x = 0; x < 128; ++x)
           if (x >= valid) sv[x] = pad;
       }
-      const float m_blk = (pos ? max128(sv) : min128(sv)) * cst;
+      const float m_blk = __int2float_rn(pos ? imax128(sv) : imin128(sv)) * cst;
       m = fmaxf(m, m_blk);
       // power-of-two reference: re-set to ceil(m) once m exceeds it by more than 8, so
       // p <= 2^8 stays below E4M3's 448 and every rescale is an exact power of two
@@ -371,7 +370,7 @@ __global__ void __launch_bounds__(320, 1) attn_qbsa_kernel(const __grid_constant
       uint32_t pk[32];
 #pragma unroll
       for (int x = 0; x < 32; ++x)
-        pk[x] = fma_exp2_e4m3x4(sv[4 * x], sv[4 * x + 1], sv[4 * x + 2], sv[4 * x + 3], cc, nr);
+        pk[x] = i2f_fma_exp2_e4m3x4(sv[4 * x], sv[4 * x + 1], sv[4 * x + 2], sv[4 * x + 3], cc, nr);
       if (valid < kTile) {  // tail block: zero the weights of keys past S_kv whatever c is
 #pragma unroll
         for (int x = 0; x < 32; ++x) {
@@ -451,7 +450,7 @@ __global__ void __launch_bounds__(320, 1) attn_qbsa_kernel(const __grid_constant
 
   tc_fence_before();
   __syncthreads();
-  if (warp == C::kWarpMma) {
+  if (warp == C::kWarpQK) {
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmemCols);
   }

@@ -447,6 +447,54 @@ __device__ __forceinline__ uint32_t fma_exp2_e4m3x4(float s0, float s1, float s2
   return r;
 }
 
+// As fma_exp2_e4m3x4, from four s32 scores (exact in f32: |s| < 2^24).
+__device__ __forceinline__ uint32_t i2f_fma_exp2_e4m3x4(uint32_t s0, uint32_t s1, uint32_t s2, uint32_t s3,
+                                                        uint64_t cc, uint64_t nr) {
+  uint32_t r;
+  asm("{\n\t.reg .f32 f0, f1, f2, f3, e0, e1, e2, e3;\n\t.reg .b64 a01, a23, z01, z23;\n\t"
+      ".reg .b32 h01, h23;\n\t.reg .b16 lo, hi;\n\t"
+      "cvt.rn.f32.s32 f0, %1;\n\t"
+      "cvt.rn.f32.s32 f1, %2;\n\t"
+      "cvt.rn.f32.s32 f2, %3;\n\t"
+      "cvt.rn.f32.s32 f3, %4;\n\t"
+      "mov.b64 a01, {f0, f1};\n\t"
+      "mov.b64 a23, {f2, f3};\n\t"
+      "fma.rn.f32x2 z01, a01, %5, %6;\n\t"
+      "fma.rn.f32x2 z23, a23, %5, %6;\n\t"
+      "mov.b64 {e0, e1}, z01;\n\t"
+      "mov.b64 {e2, e3}, z23;\n\t"
+      "ex2.approx.ftz.f32 e0, e0;\n\t"
+      "ex2.approx.ftz.f32 e1, e1;\n\t"
+      "ex2.approx.ftz.f32 e2, e2;\n\t"
+      "ex2.approx.ftz.f32 e3, e3;\n\t"
+      "cvt.rn.f16x2.f32 h01, e1, e0;\n\t"
+      "cvt.rn.f16x2.f32 h23, e3, e2;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f16x2 lo, h01;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f16x2 hi, h23;\n\t"
+      "mov.b32 %0, {lo, hi};\n\t}"
+      : "=r"(r)
+      : "r"(s0), "r"(s1), "r"(s2), "r"(s3), "l"(cc), "l"(nr));
+  return r;
+}
+
+// Maximum / minimum of 128 s32 values (two-input integer ops at full rate).
+__device__ __forceinline__ int32_t imax128(const uint32_t (&v)[128]) {
+  int32_t a[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) a[i] = static_cast<int32_t>(v[i]);
+#pragma unroll
+  for (int x = 8; x < 128; ++x) a[x & 7] = max(a[x & 7], static_cast<int32_t>(v[x]));
+  return max(max(max(a[0], a[1]), max(a[2], a[3])), max(max(a[4], a[5]), max(a[6], a[7])));
+}
+__device__ __forceinline__ int32_t imin128(const uint32_t (&v)[128]) {
+  int32_t a[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) a[i] = static_cast<int32_t>(v[i]);
+#pragma unroll
+  for (int x = 8; x < 128; ++x) a[x & 7] = min(a[x & 7], static_cast<int32_t>(v[x]));
+  return min(min(min(a[0], a[1]), min(a[2], a[3])), min(min(a[4], a[5]), min(a[6], a[7])));
+}
+
 // Three-input minimum (one instruction on sm_100).
 __device__ __forceinline__ float fmin3(float a, float b, float c) {
   float d;
