@@ -152,10 +152,6 @@ __device__ __forceinline__ DenseWork dense_work(const DenseParams& p) {
   return w;
 }
 
-__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
 template <int D>
 __global__ void __launch_bounds__(320, 1) attn_dense_kernel(const __grid_constant__ DenseParams p) {
   using C = DenseCfg<D>;

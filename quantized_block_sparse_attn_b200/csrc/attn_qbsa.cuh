@@ -11,17 +11,21 @@
 // the tensor core and take turns on the special-function unit: while one tile's
 // warps load scores and reduce row maxima, the other tile's warps are in their
 // exponentials.  Each tile's row of the block mask is first compacted into the
-// ascending list of kept key blocks in shared memory, with each block's
-// dequantisation constant s_q * s_k * scale * log2(e).  Then:
+// ascending list of kept key blocks in shared memory.  Then:
 //   warps 0..3  softmax of tile 0, warps 4..7 softmax of tile 1: one thread per query
 //               row (TMEM lane 32*(warp%4)+lane), all 128 key columns of a block.
-//               Exact s32 -> f32 (|dot| < 2^24), online softmax whose weights
-//               p = 2^(z - R) use a power-of-two reference R re-set to ceil(running
-//               max) only when the max exceeds it by more than 8 (exact power-of-two
-//               rescales of O and L, rare), P -> FP16 -> E4M3 into TMEM, epilogue
-//               O * v_scale / L -> bf16.
+//               Exact s32 -> f32 (|dot| < 2^24), dequantisation constant
+//               c = s_q * s_k * scale * log2(e) (s_k fetched a block ahead), online
+//               softmax whose weights p = 2^(z - R) use a power-of-two reference R
+//               re-set to ceil(running max) only when the max exceeds it by more than 8
+//               (exact power-of-two rescales of O and L, rare);
+//               P -> FP16 -> E4M3 into TMEM; epilogue O * v_scale / L -> bf16 staged
+//               in the tile's Q buffer (free by then) and a second buffer, written by
+//               TMA stores.
 //   warp 8      TMA producer: Q of both tiles once; K and V tiles of the kept blocks
-//               of both tiles, interleaved (t0 j, t1 j, t0 j+1, ...), 5-stage ring.
+//               of both tiles, interleaved (t0 j, t1 j, t0 j+1, ...), into a 4-stage K
+//               ring (a stage is free once its QK retired) and a 5-stage V ring (free
+//               once its P·V retired), so K is fetched about two blocks ahead.
 //   warp 9      TMEM owner + QK issuer: S = Q8_t K8ᵀ (kind::i8, s32 into the one
 //               shared S buffer) once the S buffer's previous reader is done.
 //   warp 10     PV issuer: [O_t | L_t] += P8_t [V8 | 1] as one N = 144 MMA
@@ -48,6 +52,7 @@ struct QbsaParams {
   CUtensorMap tm_q;  // 4-D {128, rows, heads, batch} int8, box {128, 128, 1, 1}, SW128
   CUtensorMap tm_k;
   CUtensorMap tm_v;  // E4M3 bytes, same geometry
+  CUtensorMap tm_o;  // bf16 output {128, Sq, Nq, B}, box {64, 128, 1, 1}, SW128
   const float* q_scale;   // [B, Nq, nqb]
   const float* k_scale;   // [B, Nkv, nkb]
   const float* v_scale;   // [B, Nkv, 128]
@@ -59,25 +64,29 @@ struct QbsaParams {
   int n_pair;             // ceil(nqb / 2) query-block pairs per (batch, head)
   int n_rank;             // B * n_pair
   int head_grp;           // query heads per L2 group
+  int mask_v16;           // mask rows are 16-byte aligned with nkb % 16 == 0 (vector compaction)
   float scale_log2;       // scale * log2(e)
 };
 
 struct QbsaCfg {
   static constexpr int D = 128;
-  static constexpr int kStages = 5;                 // (K, V) tile pairs in flight
+  static constexpr int kKStages = 4;                // K tiles in flight
+  static constexpr int kVStages = 5;                // V tiles in flight
   static constexpr int kTileBytes = kTile * 128;    // 128 rows x 128 bytes
   static constexpr int kQOff = 0;                   // Q of tile 0, then tile 1
   static constexpr int kKOff = kQOff + 2 * kTileBytes;
-  static constexpr int kVOff = kKOff + kStages * kTileBytes;
-  static constexpr int kOnesOff = kVOff + kStages * kTileBytes;   // 32 rows x 128 B of E4M3 1.0
-  static constexpr int kCOff = kOnesOff + 4096;                    // float [2][kMax] dequant constants
-  static constexpr int kListOff = kCOff + 2 * kQbsaMaxKBlocks * 4;  // uint16 [2][kMax] kept blocks
+  static constexpr int kVOff = kKOff + kKStages * kTileBytes;
+  static constexpr int kEOff = kVOff + kVStages * kTileBytes;     // [2] epilogue staging, columns 64..127
+  static constexpr int kOnesOff = kEOff + 2 * kTileBytes;           // 32 rows x 128 B of E4M3 1.0
+  static constexpr int kListOff = kOnesOff + 4096;                 // uint16 [2][kMax] kept blocks
   static constexpr int kVscOff = kListOff + 2 * kQbsaMaxKBlocks * 2;  // float [128] value scales
   static constexpr int kBarOff = kVscOff + 128 * 4;
   static constexpr int kBarQFull = 0;
-  static constexpr int kBarKVFull = 1;
-  static constexpr int kBarKVEmpty = kBarKVFull + kStages;
-  static constexpr int kBarSFull = kBarKVEmpty + kStages;  // [2], per tile
+  static constexpr int kBarKFull = 1;
+  static constexpr int kBarKEmpty = kBarKFull + kKStages;
+  static constexpr int kBarVFull = kBarKEmpty + kKStages;
+  static constexpr int kBarVEmpty = kBarVFull + kVStages;
+  static constexpr int kBarSFull = kBarVEmpty + kVStages;  // [2], per tile
   static constexpr int kBarSFree = kBarSFull + 2;          // [2], per tile
   static constexpr int kBarPFull = kBarSFree + 2;          // [2]
   static constexpr int kBarPVDone = kBarPFull + 2;         // [2]
@@ -93,8 +102,12 @@ struct QbsaCfg {
   static constexpr int kWarpProducer = 8, kWarpQK = 9, kWarpPV = 10;
 };
 static_assert(QbsaCfg::kSmemBytes <= 232448, "shared memory above the 227 KB opt-in limit");
+// TMA tiles and UMMA operands use the 128-byte swizzle, whose pattern repeats every 1024 bytes
+static_assert(QbsaCfg::kKOff % 1024 == 0 && QbsaCfg::kVOff % 1024 == 0 && QbsaCfg::kEOff % 1024 == 0 &&
+                  QbsaCfg::kOnesOff % 1024 == 0 && QbsaCfg::kTileBytes % 1024 == 0,
+              "swizzled buffers must start on 1024-byte boundaries");
 
-// Compact one row of the block mask (n_kb bytes, 1 = keep) into ascending indices.
+// Compact one row of the block mask (n_kb bytes, nonzero = keep) into ascending indices.
 // Executed by one full warp; returns the count (same value in every lane).
 __device__ __forceinline__ int compact_mask_row(const uint8_t* row, int n_kb, uint16_t* list, int lane) {
   int count = 0;
@@ -104,6 +117,48 @@ __device__ __forceinline__ int compact_mask_row(const uint8_t* row, int n_kb, ui
     const uint32_t m = __ballot_sync(0xffffffffu, keep);
     if (keep) list[count + __popc(m & ((1u << lane) - 1u))] = static_cast<uint16_t>(j);
     count += __popc(m);
+  }
+  return count;
+}
+
+// Same result for a 16-byte aligned row with n_kb % 16 == 0 and n_kb <= 2048: every lane
+// loads its 16-byte chunks at once (one memory round trip), counts the nonzero bytes,
+// and a warp prefix sum places each lane's indices.
+__device__ __forceinline__ int compact_mask_row_v16(const uint8_t* row, int n_kb, uint16_t* list, int lane) {
+  const int n_chunks = n_kb >> 4;
+  const uint4* r4 = reinterpret_cast<const uint4*>(row);
+  uint4 v[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int c = lane + 32 * i;
+    v[i] = (c < n_chunks) ? __ldg(r4 + c) : make_uint4(0u, 0u, 0u, 0u);
+  }
+  int count = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    if (32 * i >= n_chunks) break;
+    const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+    uint32_t nz[4];
+    int mine = 0;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      nz[k] = (((w[k] & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) | w[k]) & 0x80808080u;  // bit 7 of a byte: byte != 0
+      mine += __popc(nz[k]);
+    }
+    int incl = mine;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, d);
+      if (lane >= d) incl += y;
+    }
+    int pos = count + incl - mine;
+    const int j0 = (lane + 32 * i) * 16;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      for (uint32_t m = nz[k]; m != 0u; m &= m - 1u)
+        list[pos++] = static_cast<uint16_t>(j0 + 4 * k + ((__ffs(m) - 1) >> 3));
+    }
+    count += __shfl_sync(0xffffffffu, incl, 31);
   }
   return count;
 }
@@ -132,7 +187,6 @@ __global__ void __launch_bounds__(352, 1) attn_qbsa_kernel(const __grid_constant
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
   int* count_slot = reinterpret_cast<int*>(smem + C::kMiscOff + 8);  // [2]
   uint16_t* lists = reinterpret_cast<uint16_t*>(smem + C::kListOff);
-  float* csts = reinterpret_cast<float*>(smem + C::kCOff);
   float* vsc = reinterpret_cast<float*>(smem + C::kVscOff);
 
   // head groups (L2 reuse of K/V), query-block pairs in order, heads fastest in a group
@@ -148,19 +202,14 @@ __global__ void __launch_bounds__(352, 1) attn_qbsa_kernel(const __grid_constant
   const int g = h / p.group;
 
   if (warp == 0 || warp == 4) {
-    // kept-block list and dequantisation constants of tile t
+    // kept-block list of tile t
     const int t = warp >> 2;
     const int qb = 2 * pr + t;
     uint16_t* list = lists + t * kQbsaMaxKBlocks;
     int cnt = 0;
     if (qb < p.nqb) {
       const uint8_t* mrow = p.block_mask + (((int64_t)b * p.Nq + h) * p.nqb + qb) * p.nkb;
-      cnt = compact_mask_row(mrow, p.nkb, list, lane);
-      __syncwarp();
-      const float sq = p.q_scale[((int64_t)b * p.Nq + h) * p.nqb + qb];
-      const float* ks = p.k_scale + ((int64_t)b * p.Nkv + g) * p.nkb;
-      float* cst = csts + t * kQbsaMaxKBlocks;
-      for (int i = lane; i < cnt; i += 32) cst[i] = (sq * ks[list[i]]) * p.scale_log2;
+      cnt = p.mask_v16 ? compact_mask_row_v16(mrow, p.nkb, list, lane) : compact_mask_row(mrow, p.nkb, list, lane);
     }
     if (lane == 0) count_slot[t] = cnt;
   } else if (warp == 1) {
@@ -175,9 +224,13 @@ __global__ void __launch_bounds__(352, 1) attn_qbsa_kernel(const __grid_constant
     if (lane == 0) {
       *abort_flag = 0;
       mbar_init(bar(C::kBarQFull), 1);
-      for (int s = 0; s < C::kStages; ++s) {
-        mbar_init(bar(C::kBarKVFull + s), 1);
-        mbar_init(bar(C::kBarKVEmpty + s), 1);
+      for (int s = 0; s < C::kKStages; ++s) {
+        mbar_init(bar(C::kBarKFull + s), 1);
+        mbar_init(bar(C::kBarKEmpty + s), 1);
+      }
+      for (int s = 0; s < C::kVStages; ++s) {
+        mbar_init(bar(C::kBarVFull + s), 1);
+        mbar_init(bar(C::kBarVEmpty + s), 1);
       }
       for (int t = 0; t < 2; ++t) {
         mbar_init(bar(C::kBarSFull + t), 1);
@@ -219,23 +272,30 @@ __global__ void __launch_bounds__(352, 1) attn_qbsa_kernel(const __grid_constant
       for (int j = 0; ok && j < n_max; ++j) {
         for (int t = 0; t < 2; ++t) {
           if (j >= (t ? n1 : n0)) continue;
-          const int s = seq % C::kStages;
-          const uint32_t round = static_cast<uint32_t>(seq / C::kStages);
-          if (seq >= C::kStages && !mbar_wait(bar(C::kBarKVEmpty + s), (round & 1) ^ 1, abort_flag)) {
+          const int kv_row = static_cast<int>(lists[t * kQbsaMaxKBlocks + j]) * kTile;
+          const int sk = seq % C::kKStages, sv = seq % C::kVStages;
+          if (seq >= C::kKStages &&
+              !mbar_wait(bar(C::kBarKEmpty + sk), (static_cast<uint32_t>(seq / C::kKStages) & 1) ^ 1, abort_flag)) {
             ok = false;
             break;
           }
-          const int kv_row = static_cast<int>(lists[t * kQbsaMaxKBlocks + j]) * kTile;
-          mbar_arrive_expect_tx(bar(C::kBarKVFull + s), 2 * C::kTileBytes);
-          tma_load_4d(base + C::kKOff + s * C::kTileBytes, &p.tm_k, bar(C::kBarKVFull + s), 0, kv_row, g, b, pol_kv);
-          tma_load_4d(base + C::kVOff + s * C::kTileBytes, &p.tm_v, bar(C::kBarKVFull + s), 0, kv_row, g, b, pol_kv);
+          mbar_arrive_expect_tx(bar(C::kBarKFull + sk), C::kTileBytes);
+          tma_load_4d(base + C::kKOff + sk * C::kTileBytes, &p.tm_k, bar(C::kBarKFull + sk), 0, kv_row, g, b, pol_kv);
+          if (seq >= C::kVStages &&
+              !mbar_wait(bar(C::kBarVEmpty + sv), (static_cast<uint32_t>(seq / C::kVStages) & 1) ^ 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bar(C::kBarVFull + sv), C::kTileBytes);
+          tma_load_4d(base + C::kVOff + sv * C::kTileBytes, &p.tm_v, bar(C::kBarVFull + sv), 0, kv_row, g, b, pol_kv);
           ++seq;
         }
       }
       // let the copies still in flight land before the CTA can exit (matters only after an abort)
-      for (int q = max(0, seq - C::kStages); q < seq; ++q) {
-        mbar_wait_drain(bar(C::kBarKVFull + q % C::kStages), static_cast<uint32_t>(q / C::kStages) & 1);
-      }
+      for (int q = max(0, seq - C::kKStages); q < seq; ++q)
+        mbar_wait_drain(bar(C::kBarKFull + q % C::kKStages), static_cast<uint32_t>(q / C::kKStages) & 1);
+      for (int q = max(0, seq - C::kVStages); q < seq; ++q)
+        mbar_wait_drain(bar(C::kBarVFull + q % C::kVStages), static_cast<uint32_t>(q / C::kVStages) & 1);
       mbar_wait_drain(bar(C::kBarQFull), 0);
     }
   } else if (warp == C::kWarpQK) {
@@ -248,8 +308,8 @@ __global__ void __launch_bounds__(352, 1) attn_qbsa_kernel(const __grid_constant
       for (int j = 0; ok && j < n_max; ++j) {
         for (int t = 0; ok && t < 2; ++t) {
           if (j >= (t ? n1 : n0)) continue;
-          const int s = seq % C::kStages;
-          if (!mbar_wait(bar(C::kBarKVFull + s), static_cast<uint32_t>(seq / C::kStages) & 1, abort_flag) ||
+          const int s = seq % C::kKStages;
+          if (!mbar_wait(bar(C::kBarKFull + s), static_cast<uint32_t>(seq / C::kKStages) & 1, abort_flag) ||
               (prev_t >= 0 &&
                !mbar_wait(bar(C::kBarSFree + prev_t), static_cast<uint32_t>(prev_j) & 1, abort_flag))) {
             ok = false;
@@ -264,6 +324,7 @@ __global__ void __launch_bounds__(352, 1) attn_qbsa_kernel(const __grid_constant
                       idesc_qk, kk > 0 ? 1u : 0u);
           }
           mma_commit(bar(C::kBarSFull + t));
+          mma_commit(bar(C::kBarKEmpty + s));
           prev_t = t;
           prev_j = j;
           ++seq;
@@ -284,9 +345,9 @@ __global__ void __launch_bounds__(352, 1) attn_qbsa_kernel(const __grid_constant
         for (int t = 0; ok && t < 2; ++t) {
           const int nt = t ? n1 : n0;
           if (j >= nt) continue;
-          const int s = seq % C::kStages;
+          const int s = seq % C::kVStages;
           if (!mbar_wait(bar(C::kBarPFull + t), static_cast<uint32_t>(j) & 1, abort_flag) ||
-              !mbar_wait(bar(C::kBarKVFull + s), static_cast<uint32_t>(seq / C::kStages) & 1, abort_flag)) {
+              !mbar_wait(bar(C::kBarVFull + s), static_cast<uint32_t>(seq / C::kVStages) & 1, abort_flag)) {
             ok = false;
             break;
           }
@@ -303,7 +364,7 @@ __global__ void __launch_bounds__(352, 1) attn_qbsa_kernel(const __grid_constant
                       (j > 0 || kk > 0) ? 1u : 0u);
           }
           mma_commit(bar(C::kBarPVDone + t));
-          mma_commit(bar(C::kBarKVEmpty + s));
+          mma_commit(bar(C::kBarVEmpty + s));
           if (j == nt - 1) mma_commit(bar(C::kBarOFinal + t));
           ++seq;
         }
@@ -325,14 +386,21 @@ __global__ void __launch_bounds__(352, 1) attn_qbsa_kernel(const __grid_constant
     const uint32_t l_col = o_col + 128;
     const uint32_t p_col = tmem + lane_off + C::kColP + 32 * t;
     const uint16_t* list = lists + t * kQbsaMaxKBlocks;
-    const float* cst_list = csts + t * kQbsaMaxKBlocks;
+    const float* ks_row = p.k_scale + ((int64_t)b * p.Nkv + g) * p.nkb;
+    const float sq = (2 * pr + t < p.nqb ? p.q_scale[((int64_t)b * p.Nq + h) * p.nqb + 2 * pr + t] : 0.f);
+    int kb_next = nt > 0 ? list[0] : 0;
+    float ks_next = nt > 0 ? ks_row[kb_next] : 0.f;
 
     float m = kNegInf;    // running max, log2 domain
     float ref = kNegInf;  // power-of-two reference of the FP8 weights (an integer)
     bool ok = true;
     for (int j = 0; ok && j < nt; ++j) {
-      const int kb = list[j];
-      const float cst = cst_list[j];
+      const int kb = kb_next;
+      const float cst = (sq * ks_next) * p.scale_log2;
+      if (j + 1 < nt) {  // the next block's key scale, fetched while this block is processed
+        kb_next = list[j + 1];
+        ks_next = ks_row[kb_next];
+      }
       const int valid = min(kTile, p.Skv - kb * kTile);  // key columns inside S_kv
       ok = warp_wait(bar(C::kBarSFull + t), static_cast<uint32_t>(j) & 1, abort_flag);
       if (!ok) break;
@@ -404,7 +472,6 @@ __global__ void __launch_bounds__(352, 1) attn_qbsa_kernel(const __grid_constant
     }
 
     // ------------------------------------------------------------ epilogue
-    const bool row_valid = i_glob < p.Sq;
     bool have_o = ok && nt > 0;
     if (have_o) {
       // a dedicated single-use barrier: pv_done's parity cannot tell PV(n-1) from PV(n-3)
@@ -414,33 +481,47 @@ __global__ void __launch_bounds__(352, 1) attn_qbsa_kernel(const __grid_constant
     float l = 0.f;
     if (have_o) l = __uint_as_float(tmem_ld1_wait(l_col));
     const float inv_l = (l > 0.f) ? 1.0f / l : 0.f;
-    __nv_bfloat16* orow = p.out + (((int64_t)b * p.Nq + h) * p.Sq + i_glob) * 128;
+    const bool tile_live = 2 * pr + t < p.nqb;
+    // O -> bf16: columns [0,64) staged in this tile's Q buffer (its last QK has retired),
+    // columns [64,128) in a second buffer, both in the 128-byte-swizzled layout of the
+    // output tensor map, then written by two TMA stores
 #pragma unroll
-    for (int ch = 0; ch < 4; ++ch) {
-      uint32_t rr[32];
-      if (have_o) {
-        tmem_ld32_wait(o_col + ch * 32, rr);
-      } else {
+    for (int hf = 0; hf < 2; ++hf) {
+      const uint32_t stage = hf ? base + C::kEOff + t * C::kTileBytes : base + C::kQOff + t * C::kTileBytes;
 #pragma unroll
-        for (int x = 0; x < 32; ++x) rr[x] = 0u;
-      }
-      if (row_valid) {
-        uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+      for (int ch = 0; ch < 2; ++ch) {
+        uint32_t rr[32];
+        if (have_o) {
+          tmem_ld32_wait(o_col + hf * 64 + ch * 32, rr);
+        } else {
+#pragma unroll
+          for (int x = 0; x < 32; ++x) rr[x] = 0u;
+        }
 #pragma unroll
         for (int x = 0; x < 4; ++x) {
+          const int c0 = hf * 64 + ch * 32 + 8 * x;
           float f[8];
 #pragma unroll
-          for (int y = 0; y < 8; ++y) f[y] = __uint_as_float(rr[8 * x + y]) * (vsc[ch * 32 + 8 * x + y] * inv_l);
-          uint4 v;
-          v.x = pack_bf16x2(f[0], f[1]);
-          v.y = pack_bf16x2(f[2], f[3]);
-          v.z = pack_bf16x2(f[4], f[5]);
-          v.w = pack_bf16x2(f[6], f[7]);
-          dst[x] = v;
+          for (int y = 0; y < 8; ++y) f[y] = __uint_as_float(rr[8 * x + y]) * (vsc[c0 + y] * inv_l);
+          const int chunk = ch * 4 + x;  // 16-byte chunk of this row's 128-byte line
+          const uint32_t dst = stage + row * 128 + ((chunk ^ (row & 7)) << 4);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(pack_bf16x2(f[0], f[1])),
+                       "r"(pack_bf16x2(f[2], f[3])), "r"(pack_bf16x2(f[4], f[5])), "r"(pack_bf16x2(f[6], f[7]))
+                       : "memory");
         }
       }
     }
-    if (row_valid) {
+    fence_proxy_async_smem();
+    named_bar_sync(1 + t, 128);
+    if (quarter == 0 && lane == 0) {
+      if (tile_live) {
+        tma_store_4d(&p.tm_o, base + C::kQOff + t * C::kTileBytes, 0, (2 * pr + t) * kTile, h, b);
+        tma_store_4d(&p.tm_o, base + C::kEOff + t * C::kTileBytes, 64, (2 * pr + t) * kTile, h, b);
+        bulk_commit_group();
+      }
+      bulk_wait_read_all();  // shared memory must outlive the stores' reads
+    }
+    if (i_glob < p.Sq) {
       const int64_t sidx = ((int64_t)b * p.Nq + h) * p.Sq + i_glob;
       const bool live = l > 0.f;
       if (p.softmax_max) p.softmax_max[sidx] = live ? m * 0.6931471805599453f : kNegInf;
@@ -462,7 +543,9 @@ __global__ void qbsa_block_lists_kernel(const uint8_t* mask, int rows, int n_kb,
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r = blockIdx.x * 4 + warp;
   if (r >= rows) return;
-  const int cnt = compact_mask_row(mask + (int64_t)r * n_kb, n_kb, buf[warp], lane);
+  const uint8_t* row = mask + (int64_t)r * n_kb;
+  const bool v16 = (n_kb % 16 == 0) && ((reinterpret_cast<uintptr_t>(mask) & 15u) == 0);
+  const int cnt = v16 ? compact_mask_row_v16(row, n_kb, buf[warp], lane) : compact_mask_row(row, n_kb, buf[warp], lane);
   __syncwarp();
   for (int i = lane; i < n_kb; i += 32) lists[(int64_t)r * n_kb + i] = (i < cnt) ? buf[warp][i] : -1;
   if (lane == 0) counts[r] = cnt;

@@ -128,6 +128,22 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const void* map, uint3
       : "memory");
 }
 
+// Tiled TMA store from shared memory (bulk-group completion; no multicast).  Rows
+// past the tensor's extent are not written.
+__device__ __forceinline__ void tma_store_4d(const void* map, uint32_t src, int c0, int c1, int c2, int c3) {
+  asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(map),
+               "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until every committed bulk store of this thread has finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// Make this thread's generic-proxy shared-memory writes visible to the async proxy (TMA).
+__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 // ---------------------------------------------------------------------------------
 // tcgen05: TMEM allocation, MMA, commit, fences
 // ---------------------------------------------------------------------------------
@@ -475,6 +491,24 @@ __device__ __forceinline__ uint32_t i2f_fma_exp2_e4m3x4(uint32_t s0, uint32_t s1
       : "=r"(r)
       : "r"(s0), "r"(s1), "r"(s2), "r"(s3), "l"(cc), "l"(nr));
   return r;
+}
+
+// Maximum / minimum of 64 s32 values (two-input integer ops at full rate).
+__device__ __forceinline__ int32_t imax64(const uint32_t (&v)[64]) {
+  int32_t a[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) a[i] = static_cast<int32_t>(v[i]);
+#pragma unroll
+  for (int x = 8; x < 64; ++x) a[x & 7] = max(a[x & 7], static_cast<int32_t>(v[x]));
+  return max(max(max(a[0], a[1]), max(a[2], a[3])), max(max(a[4], a[5]), max(a[6], a[7])));
+}
+__device__ __forceinline__ int32_t imin64(const uint32_t (&v)[64]) {
+  int32_t a[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) a[i] = static_cast<int32_t>(v[i]);
+#pragma unroll
+  for (int x = 8; x < 64; ++x) a[x & 7] = min(a[x & 7], static_cast<int32_t>(v[x]));
+  return min(min(min(a[0], a[1]), min(a[2], a[3])), min(min(a[4], a[5]), min(a[6], a[7])));
 }
 
 // Maximum / minimum of 128 s32 values (two-input integer ops at full rate).

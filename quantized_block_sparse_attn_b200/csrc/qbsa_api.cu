@@ -374,6 +374,9 @@ qbsa_status qbsa_fwd(const int8_t* q_i8, const int8_t* k_i8, const float* q_bloc
   if ((st = make_map(&prm.tm_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, q_i8, qd, qs, 128)) != QBSA_OK) return st;
   if ((st = make_map(&prm.tm_k, CU_TENSOR_MAP_DATA_TYPE_UINT8, k_i8, kd, ks, 128)) != QBSA_OK) return st;
   if ((st = make_map(&prm.tm_v, CU_TENSOR_MAP_DATA_TYPE_UINT8, v_fp8, kd, ks, 128)) != QBSA_OK) return st;
+  const uint64_t os[3] = {256, (uint64_t)Sq * 256, (uint64_t)Nq * Sq * 256};
+  if ((st = make_map(&prm.tm_o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, attention_out, qd, os, 64)) != QBSA_OK) return st;
+  prm.mask_v16 = (nkb % 16 == 0) && aligned16(block_mask);
   if ((st = set_smem(qbsa::attn_qbsa_kernel, qbsa::QbsaCfg::kSmemBytes)) != QBSA_OK) return st;
   qbsa::attn_qbsa_kernel<<<dim3(static_cast<unsigned>(n_work)), qbsa::QbsaCfg::kThreads, qbsa::QbsaCfg::kSmemBytes,
                            static_cast<cudaStream_t>(stream)>>>(prm);
