@@ -32,6 +32,31 @@ sys.path.insert(0, ROOT)
 METRIC = "attention fwd TFLOPS (B=1,N=40,D=128) and % of B200 tensor peak vs S"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FP8_OVER_BF16 = 2.0  # nominal dense ratio (4.5 vs 2.25 PFLOP/s), applied to the measured bf16 peak
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one attn_qbsa_kernel launch from
+# one ncu capture at S=16384, keep 0.1 (profiles/attn_qbsa_kernel_S16384_keep0.1_full.md); it holds
+# only for the kernel sources it was taken on, identified by their sha1.
+QBSA_NCU_TRAFFIC = {"sources": {"quantized_block_sparse_attn_b200/csrc/attn_qbsa.cuh": "15a16c4aeb56e4a41156ee33b0decaf9112d4eca",
+                                "quantized_block_sparse_attn_b200/csrc/ptx_sm100.cuh": "00d0c231a8a4e58beb908f6eea8d5d7d9e7323ad"},
+                    "seq": 16384, "keep": 0.1, "bytes": 457652224, "alg_bytes": 420147200}
+
+
+def qbsa_traffic(seq: int, keep: float, alg_bytes: int):
+    """Per-launch DRAM traffic from the recorded ncu capture, scaled to this launch by its
+    algorithmic bytes (Q, K, V, O all grow linearly in S), or None when the kernel sources
+    changed since the capture or the keep fraction differs."""
+    import hashlib
+    rec = QBSA_NCU_TRAFFIC
+    for rel, sha in rec["sources"].items():
+        try:
+            with open(os.path.join(ROOT, rel), "rb") as f:
+                if hashlib.sha1(f.read()).hexdigest() != sha:
+                    return None, "kernel changed since the ncu capture"
+        except OSError:
+            return None, "kernel sources not found"
+    if abs(keep - rec["keep"]) > 1e-9:
+        return None, "no capture at this keep fraction"
+    return (rec["bytes"] * alg_bytes / rec["alg_bytes"],
+            f"ncu at S={rec['seq']} keep {rec['keep']}: {rec['bytes'] / 1e6:.1f} MB, scaled by algorithmic bytes")
 
 
 def parse():
@@ -323,6 +348,7 @@ def run_ours(args):
     launch_ms = sum(per_ms) / len(per_ms)
     achieved = executed / (launch_ms / 1e3) / 1e12
 
+    traffic, traffic_src = qbsa_traffic(args.seq, args.keep, alg_bytes)
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "i8xi8->s32, e4m3xe4m3->f32, bf16 out", "data": "synthetic",
@@ -332,7 +358,7 @@ def run_ours(args):
                        "dense_equivalent_tflops": world * dense_eq * args.steps / (total_ms / 1e3) / 1e12,
                        "pct_of_fp8_int8_peak": 100.0 * achieved / fp8_peak},
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": fp8_peak, "unit": "TFLOP/s",
-                         "frac": achieved / fp8_peak, "traffic": None,
+                         "frac": achieved / fp8_peak, "traffic": traffic, "traffic_source": traffic_src,
                          "peak_source": f"{peak_src} bf16 burst {bf16_peak} x {FP8_OVER_BF16} (nominal fp8/int8:bf16)",
                          "kernel": "attn_qbsa_kernel", "algorithmic_bytes": alg_bytes,
                          "hbm_gbs_algorithmic": alg_bytes / (launch_ms / 1e3) / 1e9},
