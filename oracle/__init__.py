@@ -26,9 +26,11 @@ Modules:
   pure-Python loop version for tiny inputs and the K-tile sets a tiled kernel must visit.
 * ``quant``    -- the Q/K per-block INT8 and V per-channel E4M3 quantisers and the
   quantized block-sparse forward, step by step in the article's order.
+* ``estimate`` -- block-mask estimation (block mean pooling, block scores, top-k), a plain
+  reading of the block selection the EagleQBSA article names but does not describe.
 
 Parity status of every function is stated in its docstring; none is "parity unpinned"
 except where a docstring says so.
 """
 
-from . import formats, dense, quant  # noqa: F401
+from . import formats, dense, quant, estimate  # noqa: F401
