@@ -330,6 +330,7 @@ def run_ours(args):
     peaks, peak_src = load_peaks()
     fp8_peak = peaks["bf16_tflops"] * FP8_OVER_BF16
     bf16_peak = peaks["bf16_tflops"]
+    hbm_peak = peaks["hbm_gbs"]
 
     # ---------------------------------------------------------------- main: qbsa_fwd
     inp = qbsa_inputs(args.seq, args.keep, device)
@@ -402,6 +403,9 @@ def run_ours(args):
         extra["bsa_bf16_same_mask"] = bsa_line(device, stream, inp, executed, bf16_peak, ms_step)
     del inp
     torch.cuda.empty_cache()
+    # ---------------------------------------------------------------- block-mask estimation
+    if not args.no_dense:
+        extra["mask_estimation"] = estimate_line(device, stream, args.seq, args.keep, hbm_peak)
     # ---------------------------------------------------------------- dense bf16 video workload
     if not args.no_dense:
         extra["dense_video"] = dense_line(device, stream, args.dense_seq, max(2, args.warmup), 3, bf16_peak, dist)
@@ -461,6 +465,41 @@ def bsa_line(device, stream, inp, executed, bf16_peak, qbsa_ms):
     return {"workload": f"bsa_fwd bf16 B=1 N=40 S={S} D=128, same block mask", "ms": ms,
             "executed_tflops": executed / ms / 1e9, "pct_of_bf16_peak": 100 * executed / ms / 1e9 / bf16_peak,
             "qbsa_speedup_over_bsa": ms / qbsa_ms, "kernel": "attn_dense_kernel<128> (block-mask list)"}
+
+
+def estimate_line(device, stream, S, keep, hbm_peak):
+    """Block-mask estimation (block mean pooling of Q and K, pooled scores, top-k) on the
+    quantized workload's bf16 Q/K recipe at this S."""
+    import torch
+    import quantized_block_sparse_attn_b200 as qb
+    from workloads import CONFIGS, device_blocky_qk_bf16
+    c = CONFIGS["qbsa"]
+    N, D, seed = c["Nq"], c["D"], c["seed"]
+    q = device_blocky_qk_bf16(seed, "q", 1, N, S, D, device)
+    k = device_blocky_qk_bf16(seed, "k", 1, N, S, D, device)
+    nb = -(-S // 128)
+    state = {}
+
+    def pool():
+        state["qm"] = qb.block_mean(q)
+        state["km"] = qb.block_mean(k)
+
+    def topk():
+        state["mask"] = qb.block_topk(state["qm"], state["km"], c["scale"], keep=keep)
+
+    pool_ms, _, _ = time_steps(pool, 5, 2, stream)
+    topk_ms, _, _ = time_steps(topk, 5, 2, stream)
+    qb.check(device)
+    pool_ms, topk_ms = pool_ms / 5, topk_ms / 5
+    pool_bytes = 2 * N * S * D * 2 + 2 * N * nb * D * 4  # bf16 Q and K read, fp32 means written
+    kept = int(state["mask"].sum().item())
+    del q, k, state
+    torch.cuda.empty_cache()
+    return {"workload": f"block-mask estimation B=1 N=40 S={S} D=128 keep={keep}", "ms": pool_ms + topk_ms,
+            "block_mean_ms": pool_ms, "block_mean_gbs": pool_bytes / (pool_ms / 1e3) / 1e9,
+            "block_mean_frac_of_hbm": pool_bytes / (pool_ms / 1e3) / 1e9 / hbm_peak,
+            "block_topk_ms": topk_ms, "kept_blocks": kept, "expected_kept": N * nb * qb.keep_count(nb, keep),
+            "kernels": "block_mean_kernel x2 (HBM-bound), block_topk_kernel"}
 
 
 def dense_line(device, stream, S, warmup, steps, bf16_peak, dist):

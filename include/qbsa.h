@@ -176,6 +176,35 @@ qbsa_status qbsa_block_lists(const uint8_t* block_mask, int64_t rows, int n_kb, 
                              void* stream);
 
 /*
+ * qbsa_block_mean -- first step of block-mask estimation: the mean row of every 128-token
+ * block.  The EagleQBSA article ([QBSA] 背景介绍) builds on block-sparse attention that
+ * computes only the 128x128 blocks a block mask selects (block_sparse_mask, block_shape
+ * [128, 128] in [QBSA] MindIE SD调用方式) but does not say how the mask is chosen; this
+ * library's reading pools each block to its mean row, scores block pairs by the pooled dot
+ * product and keeps the top blocks (qbsa_block_topk).
+ *   x       bf16 [B, N, S, D] contiguous (BNSD), device, 16-byte aligned; D in {64, 128, 256}.
+ *   x_mean  fp32 [B, N, ceil(S/128), D], device, caller-owned output: the mean over the
+ *           block's rows that lie inside S (a tail block averages fewer rows), summed in fp32.
+ * Asynchronous on `stream`.  QBSA_ERR_INVALID for null pointers, S < 1 or misalignment,
+ * QBSA_ERR_UNSUPPORTED for other D.
+ */
+qbsa_status qbsa_block_mean(const void* x, int B, int N, int S, int D, float* x_mean, void* stream);
+
+/*
+ * qbsa_block_topk -- second step of block-mask estimation (reading stated at
+ * qbsa_block_mean): score[b, h, i, j] = scale * <q_mean[b, h, i, :], k_mean[b, h / (Nq/Nkv), j, :]>
+ * (fp32), and block_mask[b, h, i, j] = 1 for the n_keep largest scores of each (b, h, i)
+ * row, equal scores going to the lower j; 0 elsewhere (1 = compute the block, the polarity
+ * qbsa_fwd and bsa_fwd read).
+ *   q_mean        fp32 [B, Nq, nqb, D], k_mean fp32 [B, Nkv, nkb, D] (qbsa_block_mean outputs), device.
+ *   block_mask    uint8 [B, Nq, nqb, nkb], device, caller-owned output.
+ *   block_scores  fp32 [B, Nq, nqb, nkb] or NULL: the scores, for inspection.
+ * Requires Nq % Nkv == 0, 1 <= n_keep <= nkb <= 2048, D <= 1024.  Asynchronous on `stream`.
+ */
+qbsa_status qbsa_block_topk(const float* q_mean, const float* k_mean, int B, int Nq, int Nkv, int nqb, int nkb, int D,
+                            float scale, int n_keep, uint8_t* block_mask, float* block_scores, void* stream);
+
+/*
  * qbsa_check -- waits for `stream`, then reports and clears the device error word:
  * QBSA_ERR_TIMEOUT if a kernel's bounded wait expired since the last check,
  * QBSA_ERR_CUDA on an asynchronous CUDA error, QBSA_OK otherwise.

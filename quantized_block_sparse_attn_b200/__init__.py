@@ -10,8 +10,12 @@ from ._binding import (  # noqa: F401
     QbsaError,
     attn_fwd,
     attn_tile_schedule,
+    block_mean,
+    block_topk,
     bsa_fwd,
     block_lists,
+    estimate_block_mask,
+    keep_count,
     check,
     lib,
     qbsa_fwd,

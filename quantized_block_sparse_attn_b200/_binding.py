@@ -33,6 +33,8 @@ SIGNATURES = {
     "qbsa_quantize_v": (_I, [_P, _I, _I, _I, _I, _P, _P, _P]),
     "attn_tile_schedule": (_I, [_I64, _I64, _I, _I64, _I64, _P, _P, _P, _P, _I64]),
     "qbsa_block_lists": (_I, [_P, _I64, _I, _P, _P, _P]),
+    "qbsa_block_mean": (_I, [_P, _I, _I, _I, _I, _P, _P]),
+    "qbsa_block_topk": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P, _P, _P]),
     "qbsa_check": (_I, [_P]),
     "qbsa_last_error": (ctypes.c_char_p, []),
     "qbsa_version": (_I, []),
@@ -276,3 +278,42 @@ def check(device=None):
     """Synchronise the current stream and raise if a kernel reported a device-side timeout."""
     import torch
     _ck(lib().qbsa_check(_stream(torch.device(device or "cuda:0"))))
+
+
+def block_mean(x):
+    """Mean row of every 128-token block of a BNSD bf16 device tensor -> fp32 [B, N, ceil(S/128), D]."""
+    import torch
+    B, N, S, D = x.shape
+    if x.dtype != torch.bfloat16 or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("x must be a contiguous bfloat16 CUDA tensor")
+    out = torch.empty((B, N, -(-S // 128), D), dtype=torch.float32, device=x.device)
+    _ck(lib().qbsa_block_mean(_ptr(x), B, N, S, D, _ptr(out), _stream(x.device)))
+    return out
+
+
+def keep_count(n_kb: int, keep: float) -> int:
+    """Blocks kept per query block for a keep fraction: max(1, min(n_kb, round(keep * n_kb)))."""
+    return max(1, min(n_kb, int(round(keep * n_kb))))
+
+
+def block_topk(q_mean, k_mean, scale: float, *, keep: float = None, n_keep: int = None, return_scores: bool = False):
+    """Block mask (uint8 [B, Nq, nqb, nkb], 1 = compute) keeping the n_keep best pooled scores per query block."""
+    import torch
+    B, Nq, nqb, D = q_mean.shape
+    Nkv, nkb = k_mean.shape[1], k_mean.shape[2]
+    if n_keep is None:
+        n_keep = keep_count(nkb, keep)
+    for t in (q_mean, k_mean):
+        if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("q_mean and k_mean must be contiguous float32 CUDA tensors")
+    mask = torch.empty((B, Nq, nqb, nkb), dtype=torch.uint8, device=q_mean.device)
+    scores = torch.empty((B, Nq, nqb, nkb), dtype=torch.float32, device=q_mean.device) if return_scores else None
+    _ck(lib().qbsa_block_topk(_ptr(q_mean), _ptr(k_mean), B, Nq, Nkv, nqb, nkb, D, scale, n_keep, _ptr(mask),
+                              _ptr(scores), _stream(q_mean.device)))
+    return (mask, scores) if return_scores else mask
+
+
+def estimate_block_mask(q, k, scale: float, keep: float, *, return_scores: bool = False):
+    """Block mask for block-sparse attention from bf16 BNSD Q and K: pool, score, keep the top blocks."""
+    return block_topk(block_mean(q), block_mean(k), scale, keep=keep, return_scores=return_scores)
+

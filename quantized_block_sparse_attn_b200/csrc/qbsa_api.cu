@@ -15,6 +15,7 @@
 #include "../../include/qbsa.h"
 #include "attn_dense.cuh"
 #include "attn_qbsa.cuh"
+#include "estimate.cuh"
 #include "quantize.cuh"
 #include "schedule.cuh"
 
@@ -456,6 +457,42 @@ qbsa_status qbsa_block_lists(const uint8_t* block_mask, int64_t rows, int n_kb, 
   qbsa::qbsa_block_lists_kernel<<<(unsigned)grid, 128, 0, static_cast<cudaStream_t>(stream)>>>(
       block_mask, (int)rows, n_kb, lists, counts);
   return check_launch("qbsa_block_lists_kernel launch");
+}
+
+// ------------------------------------------------------------------------------
+// block-mask estimation
+// ------------------------------------------------------------------------------
+
+qbsa_status qbsa_block_mean(const void* x, int B, int N, int S, int D, float* x_mean, void* stream) {
+  if (!x || !x_mean) return fail(QBSA_ERR_INVALID, "x and x_mean must be non-null");
+  if (!aligned16(x)) return fail(QBSA_ERR_INVALID, "x must be 16-byte aligned");
+  if (B < 1 || N < 1 || S < 1) return fail(QBSA_ERR_INVALID, "B, N, S >= 1");
+  if (D != 64 && D != 128 && D != 256) return fail(QBSA_ERR_UNSUPPORTED, "block mean supports D in {64,128,256}");
+  if (S > kMaxLen) return fail(QBSA_ERR_UNSUPPORTED, "sequence length above %lld", (long long)kMaxLen);
+  const int nb = (S + qbsa::kTile - 1) / qbsa::kTile;
+  const int64_t n_cta = (int64_t)B * N * nb;
+  if (n_cta > 0x7fffffffLL) return fail(QBSA_ERR_UNSUPPORTED, "too many blocks");
+  qbsa::block_mean_kernel<<<dim3(static_cast<unsigned>(n_cta)), qbsa::kEstThreads, 0,
+                            static_cast<cudaStream_t>(stream)>>>(static_cast<const __nv_bfloat16*>(x), S, D, nb,
+                                                                  x_mean);
+  return check_launch("block_mean_kernel launch");
+}
+
+qbsa_status qbsa_block_topk(const float* q_mean, const float* k_mean, int B, int Nq, int Nkv, int nqb, int nkb, int D,
+                            float scale, int n_keep, uint8_t* block_mask, float* block_scores, void* stream) {
+  if (!q_mean || !k_mean || !block_mask) return fail(QBSA_ERR_INVALID, "q_mean, k_mean and block_mask must be non-null");
+  if (B < 1 || Nq < 1 || Nkv < 1 || nqb < 1 || nkb < 1 || D < 1) return fail(QBSA_ERR_INVALID, "sizes must be >= 1");
+  if (Nq % Nkv != 0) return fail(QBSA_ERR_INVALID, "Nq (%d) must be a multiple of Nkv (%d)", Nq, Nkv);
+  if (nkb > qbsa::kTopkMaxKBlocks) return fail(QBSA_ERR_UNSUPPORTED, "nkb above %d", qbsa::kTopkMaxKBlocks);
+  if (D > 1024) return fail(QBSA_ERR_UNSUPPORTED, "D above 1024");
+  if (n_keep < 1 || n_keep > nkb) return fail(QBSA_ERR_INVALID, "n_keep must be in [1, nkb]");
+  if (!std::isfinite(scale)) return fail(QBSA_ERR_INVALID, "scale must be finite");
+  const int64_t n_cta = (int64_t)B * Nq * nqb;
+  if (n_cta > 0x7fffffffLL) return fail(QBSA_ERR_UNSUPPORTED, "too many query blocks");
+  qbsa::block_topk_kernel<<<dim3(static_cast<unsigned>(n_cta)), qbsa::kTopkThreads, 0,
+                            static_cast<cudaStream_t>(stream)>>>(q_mean, k_mean, Nq, Nq / Nkv, nqb, nkb, D, scale,
+                                                                  n_keep, block_mask, block_scores);
+  return check_launch("block_topk_kernel launch");
 }
 
 qbsa_status qbsa_check(void* stream) {

@@ -103,6 +103,26 @@ def test_qbsa_fwd_rejects_before_launch():
     assert L.qbsa_fwd(*bad) == 2
 
 
+def test_block_estimation_rejects_before_launch():
+    fake = ctypes.c_void_p(0x10000)
+    L = qb.lib()
+    assert L.qbsa_block_mean(fake, 1, 2, 300, 96, fake, None) == 2           # D not in {64, 128, 256}
+    assert L.qbsa_block_mean(None, 1, 2, 300, 128, fake, None) == 1
+    assert L.qbsa_block_mean(ctypes.c_void_p(0x10008), 1, 2, 300, 128, fake, None) == 1  # misaligned
+    args = [fake, fake, 1, 4, 2, 3, 512, 128, 0.1, 51, fake, None, None]
+    bad = list(args)
+    bad[9] = 0                                                                # n_keep < 1
+    assert L.qbsa_block_topk(*bad) == 1
+    bad[9] = 513                                                              # n_keep > nkb
+    assert L.qbsa_block_topk(*bad) == 1
+    bad = list(args)
+    bad[4] = 3                                                                # Nq % Nkv != 0
+    assert L.qbsa_block_topk(*bad) == 1
+    bad = list(args)
+    bad[6] = 4096                                                             # nkb above 2048
+    assert L.qbsa_block_topk(*bad) == 2
+
+
 SCHED_CASES = [
     (256, 256, 0, INF, INF), (300, 500, 0, INF, INF), (1000, 1000, 2, INF, INF), (1000, 777, 2, INF, INF),
     (777, 1000, 3, INF, INF), (1000, 777, 3, INF, INF), (129, 1, 3, INF, INF), (1, 129, 3, INF, INF),
