@@ -199,7 +199,8 @@ qbsa_status qbsa_block_mean(const void* x, int B, int N, int S, int D, float* x_
  *   q_mean        fp32 [B, Nq, nqb, D], k_mean fp32 [B, Nkv, nkb, D] (qbsa_block_mean outputs), device.
  *   block_mask    uint8 [B, Nq, nqb, nkb], device, caller-owned output.
  *   block_scores  fp32 [B, Nq, nqb, nkb] or NULL: the scores, for inspection.
- * Requires Nq % Nkv == 0, 1 <= n_keep <= nkb <= 2048, D <= 1024.  Asynchronous on `stream`.
+ * Requires Nq % Nkv == 0, 1 <= n_keep <= nkb <= 2048, D a multiple of 4 and <= 1024, k_mean
+ * 16-byte aligned.  Asynchronous on `stream`.
  */
 qbsa_status qbsa_block_topk(const float* q_mean, const float* k_mean, int B, int Nq, int Nkv, int nqb, int nkb, int D,
                             float scale, int n_keep, uint8_t* block_mask, float* block_scores, void* stream);

@@ -58,72 +58,96 @@ __global__ void __launch_bounds__(kEstThreads) block_mean_kernel(const __nv_bflo
   }
 }
 
-// Orderable 64-bit sort key: ascending key = descending score, then ascending index.
-__device__ __forceinline__ uint64_t topk_key(float s, int j) {
-  const uint32_t u = __float_as_uint(s);
-  const uint32_t up = (u & 0x80000000u) ? ~u : (u | 0x80000000u);  // ascending with the score
-  return (static_cast<uint64_t>(~up) << 32) | static_cast<uint32_t>(j);
+// Orderable score key: unsigned order equals the order of the scores (-0 taken as +0).
+__device__ __forceinline__ uint32_t score_key(float s) {
+  const uint32_t u = __float_as_uint(s + 0.0f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// One CTA per (b, h, query block): scores of all key blocks of kv head h / group, a bitonic
-// sort of the (score, index) keys in shared memory, and the mask row (1 = compute).
+// Query blocks per CTA of block_topk_kernel: the pooled key matrix of a head is read once per
+// group of this many query blocks.
+constexpr int kTopkGroup = 8;
+__host__ inline int topk_smem_bytes(int nkb, int D) { return kTopkGroup * (D + nkb) * 4; }
+
+// One CTA per (b, h, group of kTopkGroup query blocks).
+// Phase 1: thread j' owns key rows j = j' + 256 k and scores each against every pooled query of
+//          the group (the queries sit in shared memory and are read as broadcasts).
+// Phase 2: warp u selects for query block u: the n_keep-th largest score key v is found bit by
+//          bit (32 counting passes), every key > v is kept, and the remaining places go to the
+//          keys equal to v in ascending block order; the mask row is written (1 = compute).
 __global__ void __launch_bounds__(kTopkThreads) block_topk_kernel(const float* __restrict__ qm,
                                                                   const float* __restrict__ km, int Nq, int group,
                                                                   int nqb, int nkb, int D, float scale, int n_keep,
                                                                   uint8_t* __restrict__ mask,
                                                                   float* __restrict__ scores) {
-  __shared__ uint64_t keys[kTopkMaxKBlocks];
-  __shared__ uint8_t sel[kTopkMaxKBlocks];
-  __shared__ float qrow[1024];
-  const int i = blockIdx.x % nqb;
-  const int64_t bh = blockIdx.x / nqb;  // b * Nq + h
+  extern __shared__ __align__(16) uint8_t topk_smem[];
+  float* qrows = reinterpret_cast<float*>(topk_smem);                              // [group][D]
+  uint32_t* keys = reinterpret_cast<uint32_t*>(topk_smem + kTopkGroup * D * 4);    // [group][nkb]
+  const int n_grp = (nqb + kTopkGroup - 1) / kTopkGroup;
+  const int i0 = (blockIdx.x % n_grp) * kTopkGroup;
+  const int nq = min(kTopkGroup, nqb - i0);
+  const int64_t bh = blockIdx.x / n_grp;  // b * Nq + h
   const int h = static_cast<int>(bh % Nq);
   const int64_t b = bh / Nq;
   const int64_t bg = b * (Nq / group) + h / group;
-  for (int d = threadIdx.x; d < D; d += kTopkThreads) qrow[d] = qm[(bh * nqb + i) * D + d];
-  int npow = 1;
-  while (npow < nkb) npow <<= 1;
-  for (int j = threadIdx.x; j < npow; j += kTopkThreads) {
-    keys[j] = ~0ull;  // padding sorts last
-    if (j < nkb) sel[j] = 0;
+  for (int e = threadIdx.x; e < kTopkGroup * D; e += kTopkThreads) {
+    const int u = e / D;
+    qrows[e] = (u < nq) ? qm[(bh * nqb + i0 + u) * D + (e - u * D)] : 0.f;
   }
   __syncthreads();
-  // warp-cooperative dot products: lanes split the channels, a shuffle tree sums them
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const float* kbase = km + bg * nkb * D;
-  for (int j = warp; j < nkb; j += kTopkThreads / 32) {
-    float s = 0.f;
-    for (int d = lane; d < D; d += 32) s = fmaf(qrow[d], kbase[(int64_t)j * D + d], s);
+  const int d4n = D >> 2;
+  for (int j = threadIdx.x; j < nkb; j += kTopkThreads) {
+    const float4* krow = reinterpret_cast<const float4*>(kbase + (int64_t)j * D);
+    float s[kTopkGroup];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    s *= scale;
-    if (lane == 0) {
-      keys[j] = topk_key(s, j);
-      if (scores) scores[(bh * nqb + i) * nkb + j] = s;
-    }
-  }
-  __syncthreads();
-  // bitonic sort, ascending, over npow keys
-  for (int k = 2; k <= npow; k <<= 1) {
-    for (int jj = k >> 1; jj > 0; jj >>= 1) {
-      for (int t = threadIdx.x; t < npow; t += kTopkThreads) {
-        const int p = t ^ jj;
-        if (p > t) {
-          const uint64_t a = keys[t], c = keys[p];
-          const bool up = (t & k) == 0;
-          if ((a > c) == up) {
-            keys[t] = c;
-            keys[p] = a;
-          }
-        }
+    for (int u = 0; u < kTopkGroup; ++u) s[u] = 0.f;
+    for (int d4 = 0; d4 < d4n; ++d4) {
+      const float4 kv = __ldg(krow + d4);
+#pragma unroll
+      for (int u = 0; u < kTopkGroup; ++u) {
+        const float4 qv = reinterpret_cast<const float4*>(qrows + u * D)[d4];
+        s[u] = fmaf(qv.w, kv.w, fmaf(qv.z, kv.z, fmaf(qv.y, kv.y, fmaf(qv.x, kv.x, s[u]))));
       }
-      __syncthreads();
+    }
+#pragma unroll
+    for (int u = 0; u < kTopkGroup; ++u) {
+      if (u < nq) {
+        const float sc = s[u] * scale;
+        keys[u * nkb + j] = score_key(sc);
+        if (scores) scores[(bh * nqb + i0 + u) * nkb + j] = sc;
+      }
     }
   }
-  for (int r = threadIdx.x; r < n_keep; r += kTopkThreads) sel[static_cast<uint32_t>(keys[r])] = 1;
   __syncthreads();
-  uint8_t* mrow = mask + (bh * nqb + i) * nkb;
-  for (int j = threadIdx.x; j < nkb; j += kTopkThreads) mrow[j] = sel[j];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int u = warp; u < nq; u += kTopkThreads / 32) {
+    const uint32_t* kr = keys + u * nkb;
+    // largest v with #{key >= v} >= n_keep, one bit at a time from the top
+    uint32_t v = 0;
+    for (int bit = 31; bit >= 0; --bit) {
+      const uint32_t cand = v | (1u << bit);
+      int c = 0;
+      for (int j = lane; j < nkb; j += 32) c += (kr[j] >= cand) ? 1 : 0;
+      c = __reduce_add_sync(0xffffffffu, c);
+      if (c >= n_keep) v = cand;
+    }
+    int above = 0;
+    for (int j = lane; j < nkb; j += 32) above += (kr[j] > v) ? 1 : 0;
+    above = __reduce_add_sync(0xffffffffu, above);
+    int ties_left = n_keep - above;  // keys equal to v still to keep, lowest block index first
+    uint8_t* mrow = mask + (bh * nqb + i0 + u) * nkb;
+    for (int j0 = 0; j0 < nkb; j0 += 32) {
+      const int j = j0 + lane;
+      const uint32_t key = (j < nkb) ? kr[j] : 0u;
+      const bool tie = (j < nkb) && key == v;
+      const uint32_t tb = __ballot_sync(0xffffffffu, tie);
+      const int before = __popc(tb & ((1u << lane) - 1u));
+      const bool keep = (j < nkb) && (key > v || (tie && before < ties_left));
+      if (j < nkb) mrow[j] = keep ? 1 : 0;
+      ties_left -= __popc(tb);
+    }
+  }
 }
 
 }  // namespace qbsa

@@ -484,12 +484,16 @@ qbsa_status qbsa_block_topk(const float* q_mean, const float* k_mean, int B, int
   if (B < 1 || Nq < 1 || Nkv < 1 || nqb < 1 || nkb < 1 || D < 1) return fail(QBSA_ERR_INVALID, "sizes must be >= 1");
   if (Nq % Nkv != 0) return fail(QBSA_ERR_INVALID, "Nq (%d) must be a multiple of Nkv (%d)", Nq, Nkv);
   if (nkb > qbsa::kTopkMaxKBlocks) return fail(QBSA_ERR_UNSUPPORTED, "nkb above %d", qbsa::kTopkMaxKBlocks);
-  if (D > 1024) return fail(QBSA_ERR_UNSUPPORTED, "D above 1024");
+  if (D > 1024 || D % 4 != 0) return fail(QBSA_ERR_UNSUPPORTED, "D must be a multiple of 4, at most 1024");
+  if (!aligned16(k_mean)) return fail(QBSA_ERR_INVALID, "k_mean must be 16-byte aligned");
   if (n_keep < 1 || n_keep > nkb) return fail(QBSA_ERR_INVALID, "n_keep must be in [1, nkb]");
   if (!std::isfinite(scale)) return fail(QBSA_ERR_INVALID, "scale must be finite");
-  const int64_t n_cta = (int64_t)B * Nq * nqb;
+  const int64_t n_cta = (int64_t)B * Nq * ((nqb + qbsa::kTopkGroup - 1) / qbsa::kTopkGroup);
   if (n_cta > 0x7fffffffLL) return fail(QBSA_ERR_UNSUPPORTED, "too many query blocks");
-  qbsa::block_topk_kernel<<<dim3(static_cast<unsigned>(n_cta)), qbsa::kTopkThreads, 0,
+  const int smem = qbsa::topk_smem_bytes(nkb, D);
+  qbsa_status st;
+  if ((st = set_smem(qbsa::block_topk_kernel, smem)) != QBSA_OK) return st;
+  qbsa::block_topk_kernel<<<dim3(static_cast<unsigned>(n_cta)), qbsa::kTopkThreads, smem,
                             static_cast<cudaStream_t>(stream)>>>(q_mean, k_mean, Nq, Nq / Nkv, nqb, nkb, D, scale,
                                                                   n_keep, block_mask, block_scores);
   return check_launch("block_topk_kernel launch");
