@@ -22,3 +22,5 @@ from ._binding import (  # noqa: F401
     quantize_qk,
     quantize_v,
 )
+
+from . import ulysses  # noqa: F401,E402  (sequence-parallel wrapper over torch.distributed)
