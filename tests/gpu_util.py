@@ -39,7 +39,16 @@ def compare_out(got: np.ndarray, ref: np.ndarray, max_abs: float, mean_abs: floa
     return mx, mn
 
 
-def compare_stats(gmax: np.ndarray, gsum: np.ndarray, rmax: np.ndarray, rsum: np.ndarray):
+# Quantized path only: a weight's FP16 and then E4M3 rounding is decided on 2^z computed by
+# ex2.approx on the GPU and exactly in the oracle, so in rare rows one weight lands on the
+# other side of an E4M3 rounding boundary.  softmax_sum is expressed against the row
+# maximum (whose weight is ~1), so such a flip moves it by at most one E4M3 step of a weight
+# <= 1, i.e. 1/8.  Those rows are allowed, up to this fraction of the rows.
+E4M3_FLIP_ABS = 0.13
+E4M3_FLIP_ROWS = 1e-3
+
+
+def compare_stats(gmax: np.ndarray, gsum: np.ndarray, rmax: np.ndarray, rsum: np.ndarray, e4m3_flips: bool = False):
     sel = ~np.isnan(rmax)
     gm, gs, rm, rs = gmax[sel], gsum[sel], rmax[sel], rsum[sel]
     dead = np.isneginf(rm)
@@ -47,4 +56,12 @@ def compare_stats(gmax: np.ndarray, gsum: np.ndarray, rmax: np.ndarray, rsum: np
     assert np.all(gs[dead] == 0)
     live = ~dead
     assert np.all(np.abs(gm[live] - rm[live]) <= STAT_MAX_RTOL * np.maximum(1.0, np.abs(rm[live])))
-    assert np.all(np.abs(gs[live] - rs[live]) <= STAT_SUM_RTOL * np.abs(rs[live]))
+    err = np.abs(gs[live] - rs[live])
+    bad = err > STAT_SUM_RTOL * np.abs(rs[live])
+    if not e4m3_flips:
+        assert not bad.any(), f"{bad.sum()} rows: softmax_sum off by up to {err.max():.3e}"
+        return
+    n_bad, n_live = int(bad.sum()), int(live.sum())
+    print(f"softmax_sum: {n_bad} of {n_live} rows beyond {STAT_SUM_RTOL} relative, max abs {err.max():.3e}")
+    assert np.all(err <= E4M3_FLIP_ABS), f"softmax_sum off by {err.max():.3e} (more than one E4M3 step)"
+    assert n_bad <= max(1, E4M3_FLIP_ROWS * n_live), f"{n_bad} of {n_live} rows beyond {STAT_SUM_RTOL}"

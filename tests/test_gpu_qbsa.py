@@ -71,6 +71,26 @@ def test_qbsa_unequal_tile_pairs(sign):
     compare_stats(gmax, gsum, rmax, rsum)
 
 
+@pytest.mark.parametrize("sign", [1.0, -1.0])
+def test_qbsa_many_units_per_cta(sign):
+    """More query-block pairs than SMs, so every CTA of the persistent grid walks several
+    (head, pair) units back to back: ragged lengths, GQA, empty and unequal mask rows."""
+    B, Nq, Nkv, Sq, Skv, D = 2, 40, 8, 1000, 777, 128
+    nqb, nkb = 8, 7
+    q = iid_normal_bf16(24, 0, B, Nq, Sq, D)
+    k = iid_normal_bf16(24, 1, B, Nkv, Skv, D)
+    v = iid_normal_bf16(24, 2, B, Nkv, Skv, D)
+    q8, qs, k8, ks, v8, vs = _quantized(q, k, v)
+    bm = (random_atten_mask(24, (B, Nq, nqb, nkb), 0.6) == 0).astype(np.uint8)
+    bm[0, 3, :, :] = 0          # a head with no kept block at all
+    bm[1, 7, 2, :] = 0
+    scale = sign * D ** -0.5
+    got, gmax, gsum = _run(q8, qs, k8, ks, v8, vs, bm, scale)
+    ref, rmax, rsum = quant.qbsa_forward(q8, k8, qs, ks, v8, vs, bm, scale)
+    compare_out(got, ref, QUANT_MAX_ABS)
+    compare_stats(gmax, gsum, rmax, rsum, e4m3_flips=True)
+
+
 def test_qbsa_short_loops_repeated():
     """Two or three kept blocks per query block, repeated: the last-P·V wait must not pass early."""
     D = 128
