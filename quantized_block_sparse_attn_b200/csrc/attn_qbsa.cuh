@@ -94,7 +94,7 @@ struct QbsaCfg {
   static constexpr int kBarDrain = kBarOFinal + 2;         // [2] single use: every MMA of an issuer retired
   static constexpr int kNumBars = kBarDrain + 2;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // tmem addr, abort flag, counts[2]
-  static constexpr int kSmemBytes = kMiscOff + 16 + 1024;
+  static constexpr int kSmemBytes = kMiscOff + 32 + 1024;
   static constexpr uint32_t kTmemCols = 512;
   // O_t|L_t at kColO[t] (L_t = its column 128), P_t at kColP + 32 t
   static constexpr uint32_t kColO0 = 0, kColS = 160, kColO1 = 288, kColP = 448;
@@ -186,6 +186,7 @@ __global__ void __launch_bounds__(352, 1) attn_qbsa_kernel(const __grid_constant
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
   int* count_slot = reinterpret_cast<int*>(smem + C::kMiscOff + 8);  // [2]
+  volatile int* qk_issued = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 16);  // [2] QKs issued per tile
   uint16_t* lists = reinterpret_cast<uint16_t*>(smem + C::kListOff);
   float* vsc = reinterpret_cast<float*>(smem + C::kVscOff);
 
@@ -223,6 +224,8 @@ __global__ void __launch_bounds__(352, 1) attn_qbsa_kernel(const __grid_constant
   } else if (warp == C::kWarpProducer) {
     if (lane == 0) {
       *abort_flag = 0;
+      qk_issued[0] = 0;
+      qk_issued[1] = 0;
       mbar_init(bar(C::kBarQFull), 1);
       for (int s = 0; s < C::kKStages; ++s) {
         mbar_init(bar(C::kBarKFull + s), 1);
@@ -325,6 +328,7 @@ __global__ void __launch_bounds__(352, 1) attn_qbsa_kernel(const __grid_constant
           }
           mma_commit(bar(C::kBarSFull + t));
           mma_commit(bar(C::kBarKEmpty + s));
+          qk_issued[t] = j + 1;  // lets the PV issuer queue behind this QK (see there)
           prev_t = t;
           prev_j = j;
           ++seq;
@@ -346,6 +350,12 @@ __global__ void __launch_bounds__(352, 1) attn_qbsa_kernel(const __grid_constant
           const int nt = t ? n1 : n0;
           if (j >= nt) continue;
           const int s = seq % C::kVStages;
+          // QK_t(j+1) is on the softmax's critical path and this P·V is not (its P buffer is
+          // reused only a block later): let that QK reach the tensor core first, as a single
+          // issuer would order them (bounded; the order never affects results)
+          if (j + 1 < nt) {
+            for (int spin = 0; spin < 4096 && qk_issued[t] < j + 2 && !*abort_flag; ++spin) __nanosleep(32);
+          }
           if (!mbar_wait(bar(C::kBarPFull + t), static_cast<uint32_t>(j) & 1, abort_flag) ||
               !mbar_wait(bar(C::kBarVFull + s), static_cast<uint32_t>(seq / C::kVStages) & 1, abort_flag)) {
             ok = false;
