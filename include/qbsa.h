@@ -206,6 +206,16 @@ qbsa_status qbsa_block_topk(const float* q_mean, const float* k_mean, int B, int
                             float scale, int n_keep, uint8_t* block_mask, float* block_scores, void* stream);
 
 /*
+ * qbsa_wait_selftest -- test hook for failure detection (no counterpart on the source
+ * pages): launches one thread that waits, through the same bounded mbarrier wait every
+ * kernel of this library uses, on a phase that nothing ever completes.  After the wait
+ * limit (2 s) the thread records a timeout in the device error word and the kernel ends
+ * normally, so the next qbsa_check(stream) returns QBSA_ERR_TIMEOUT and the context stays
+ * usable.  No fault, trap or endless loop is involved.
+ */
+qbsa_status qbsa_wait_selftest(void* stream);
+
+/*
  * qbsa_check -- waits for `stream`, then reports and clears the device error word:
  * QBSA_ERR_TIMEOUT if a kernel's bounded wait expired since the last check,
  * QBSA_ERR_CUDA on an asynchronous CUDA error, QBSA_OK otherwise.

@@ -35,6 +35,7 @@ SIGNATURES = {
     "qbsa_block_lists": (_I, [_P, _I64, _I, _P, _P, _P]),
     "qbsa_block_mean": (_I, [_P, _I, _I, _I, _I, _P, _P]),
     "qbsa_block_topk": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P, _P, _P]),
+    "qbsa_wait_selftest": (_I, [_P]),
     "qbsa_check": (_I, [_P]),
     "qbsa_last_error": (ctypes.c_char_p, []),
     "qbsa_version": (_I, []),

@@ -499,6 +499,27 @@ qbsa_status qbsa_block_topk(const float* q_mean, const float* k_mean, int B, int
   return check_launch("block_topk_kernel launch");
 }
 
+namespace qbsa {
+// Failure-detection self-test: one thread waits, through the kernels' own bounded wait, on
+// an mbarrier phase that nothing completes; the wait gives up after its time limit, records
+// the timeout in the device error word and the kernel returns normally.
+__global__ void wait_selftest_kernel() {
+  __shared__ uint64_t barrier;
+  __shared__ int abort_flag;
+  if (threadIdx.x != 0) return;
+  abort_flag = 0;
+  const uint32_t bar = smem_u32(&barrier);
+  mbar_init(bar, 1);
+  fence_mbar_init();
+  mbar_wait(bar, 0, &abort_flag);  // no arrival ever comes
+}
+}  // namespace qbsa
+
+qbsa_status qbsa_wait_selftest(void* stream) {
+  qbsa::wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>();
+  return check_launch("wait_selftest_kernel launch");
+}
+
 qbsa_status qbsa_check(void* stream) {
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
