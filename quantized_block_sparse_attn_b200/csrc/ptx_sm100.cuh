@@ -272,31 +272,6 @@ __device__ __forceinline__ void tmem_ld64_wait(uint32_t taddr, uint32_t (&r)[64]
       : "memory");
 }
 
-// Issue a load of 64 consecutive 32-bit columns without waiting.  The registers are
-// undefined until tmem_ld64_wait(r) on the same array; that wait takes them as
-// read-write operands, so no use of them can be scheduled before it.
-__device__ __forceinline__ void tmem_ld64_issue(uint32_t taddr, uint32_t (&r)[64]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,"
-      "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
-      "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];"
-      : QBSA_R8(0), QBSA_R8(8), QBSA_R8(16), QBSA_R8(24), QBSA_R8(32), QBSA_R8(40), QBSA_R8(48), QBSA_R8(56)
-      : "r"(taddr)
-      : "memory");
-}
-#define QBSA_RW8(i) "+r"(r[i]), "+r"(r[i + 1]), "+r"(r[i + 2]), "+r"(r[i + 3]), "+r"(r[i + 4]), "+r"(r[i + 5]), \
-                    "+r"(r[i + 6]), "+r"(r[i + 7])
-__device__ __forceinline__ void tmem_ld64_wait(uint32_t (&r)[64]) {
-  asm volatile("tcgen05.wait::ld.sync.aligned;"
-               : QBSA_RW8(0), QBSA_RW8(8), QBSA_RW8(16), QBSA_RW8(24), QBSA_RW8(32), QBSA_RW8(40), QBSA_RW8(48),
-                 QBSA_RW8(56)
-               :
-               : "memory");
-}
-#undef QBSA_RW8
-
 // Load 128 consecutive 32-bit columns (two 64-column loads, one wait).
 __device__ __forceinline__ void tmem_ld128_wait(uint32_t taddr, uint32_t (&r)[128]) {
   asm volatile(
@@ -315,13 +290,6 @@ __device__ __forceinline__ void tmem_ld128_wait(uint32_t taddr, uint32_t (&r)[12
         QBSA_R8(64), QBSA_R8(72), QBSA_R8(80), QBSA_R8(88), QBSA_R8(96), QBSA_R8(104), QBSA_R8(112), QBSA_R8(120)
       : "r"(taddr), "r"(taddr + 64)
       : "memory");
-}
-
-// Store 8 consecutive 32-bit columns (issue only; pair with tmem_st_wait).
-__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
-               "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
-               : "memory");
 }
 
 // Load one 32-bit column (lane = thread) and wait.
@@ -345,13 +313,7 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       QBSA_W8(0), QBSA_W8(8), QBSA_W8(16), QBSA_W8(24)
       : "memory");
 }
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
-      QBSA_W8(0), QBSA_W8(8)
-      : "memory");
-}
+
 __device__ __forceinline__ void tmem_st1(uint32_t taddr, uint32_t v) {
   asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(v) : "memory");
 }
@@ -397,69 +359,10 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
-// Four f32 -> four E4M3 bytes (byte i = value i), round to nearest even, saturating.
-__device__ __forceinline__ uint32_t pack_e4m3x4(float a0, float a1, float a2, float a3) {
-  uint32_t r;
-  asm("{\n\t.reg .b16 lo, hi;\n\t"
-      "cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n\t"
-      "cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n\t"
-      "mov.b32 %0, {lo, hi};\n\t}"
-      : "=r"(r)
-      : "f"(a0), "f"(a1), "f"(a2), "f"(a3));
-  return r;
-}
-
-// Four exponents x (log2 units) -> 2^x (fp32 ex2) rounded to FP16 -> four E4M3 bytes
-// (byte i = value i); both roundings nearest even, the second saturating.
-__device__ __forceinline__ uint32_t exp2_e4m3x4(float x0, float x1, float x2, float x3) {
-  uint32_t r;
-  asm("{\n\t.reg .f32 e0, e1, e2, e3;\n\t.reg .b32 h01, h23;\n\t.reg .b16 lo, hi;\n\t"
-      "ex2.approx.ftz.f32 e0, %1;\n\t"
-      "ex2.approx.ftz.f32 e1, %2;\n\t"
-      "ex2.approx.ftz.f32 e2, %3;\n\t"
-      "ex2.approx.ftz.f32 e3, %4;\n\t"
-      "cvt.rn.f16x2.f32 h01, e1, e0;\n\t"
-      "cvt.rn.f16x2.f32 h23, e3, e2;\n\t"
-      "cvt.rn.satfinite.e4m3x2.f16x2 lo, h01;\n\t"
-      "cvt.rn.satfinite.e4m3x2.f16x2 hi, h23;\n\t"
-      "mov.b32 %0, {lo, hi};\n\t}"
-      : "=r"(r)
-      : "f"(x0), "f"(x1), "f"(x2), "f"(x3));
-  return r;
-}
-
 // Two f32 in one 64-bit register pair (lo = element 0), for the packed f32x2 ops.
 __device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
   uint64_t r;
   asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-
-// Four scores s (exact integers held in f32) -> z = s * c - R with two packed
-// fma.rn.f32x2 (cc = {c, c}, nr = {-R, -R}) -> 2^z (fp32 ex2) rounded to FP16 -> four
-// E4M3 bytes (byte i = value i); both roundings nearest even, the second saturating.
-__device__ __forceinline__ uint32_t fma_exp2_e4m3x4(float s0, float s1, float s2, float s3, uint64_t cc,
-                                                    uint64_t nr) {
-  uint32_t r;
-  asm("{\n\t.reg .f32 e0, e1, e2, e3;\n\t.reg .b64 a01, a23, z01, z23;\n\t.reg .b32 h01, h23;\n\t"
-      ".reg .b16 lo, hi;\n\t"
-      "mov.b64 a01, {%1, %2};\n\t"
-      "mov.b64 a23, {%3, %4};\n\t"
-      "fma.rn.f32x2 z01, a01, %5, %6;\n\t"
-      "fma.rn.f32x2 z23, a23, %5, %6;\n\t"
-      "mov.b64 {e0, e1}, z01;\n\t"
-      "mov.b64 {e2, e3}, z23;\n\t"
-      "ex2.approx.ftz.f32 e0, e0;\n\t"
-      "ex2.approx.ftz.f32 e1, e1;\n\t"
-      "ex2.approx.ftz.f32 e2, e2;\n\t"
-      "ex2.approx.ftz.f32 e3, e3;\n\t"
-      "cvt.rn.f16x2.f32 h01, e1, e0;\n\t"
-      "cvt.rn.f16x2.f32 h23, e3, e2;\n\t"
-      "cvt.rn.satfinite.e4m3x2.f16x2 lo, h01;\n\t"
-      "cvt.rn.satfinite.e4m3x2.f16x2 hi, h23;\n\t"
-      "mov.b32 %0, {lo, hi};\n\t}"
-      : "=r"(r)
-      : "f"(s0), "f"(s1), "f"(s2), "f"(s3), "l"(cc), "l"(nr));
   return r;
 }
 
@@ -493,24 +396,6 @@ __device__ __forceinline__ uint32_t i2f_fma_exp2_e4m3x4(uint32_t s0, uint32_t s1
   return r;
 }
 
-// Maximum / minimum of 64 s32 values (two-input integer ops at full rate).
-__device__ __forceinline__ int32_t imax64(const uint32_t (&v)[64]) {
-  int32_t a[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) a[i] = static_cast<int32_t>(v[i]);
-#pragma unroll
-  for (int x = 8; x < 64; ++x) a[x & 7] = max(a[x & 7], static_cast<int32_t>(v[x]));
-  return max(max(max(a[0], a[1]), max(a[2], a[3])), max(max(a[4], a[5]), max(a[6], a[7])));
-}
-__device__ __forceinline__ int32_t imin64(const uint32_t (&v)[64]) {
-  int32_t a[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) a[i] = static_cast<int32_t>(v[i]);
-#pragma unroll
-  for (int x = 8; x < 64; ++x) a[x & 7] = min(a[x & 7], static_cast<int32_t>(v[x]));
-  return min(min(min(a[0], a[1]), min(a[2], a[3])), min(min(a[4], a[5]), min(a[6], a[7])));
-}
-
 // Maximum / minimum of 128 s32 values (two-input integer ops at full rate).
 __device__ __forceinline__ int32_t imax128(const uint32_t (&v)[128]) {
   int32_t a[8];
@@ -527,39 +412,6 @@ __device__ __forceinline__ int32_t imin128(const uint32_t (&v)[128]) {
 #pragma unroll
   for (int x = 8; x < 128; ++x) a[x & 7] = min(a[x & 7], static_cast<int32_t>(v[x]));
   return min(min(min(a[0], a[1]), min(a[2], a[3])), min(min(a[4], a[5]), min(a[6], a[7])));
-}
-
-// Three-input minimum (one instruction on sm_100).
-__device__ __forceinline__ float fmin3(float a, float b, float c) {
-  float d;
-  asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-  return d;
-}
-
-// Maximum / minimum of 128 values as trees of three-input ops (64 instructions).
-__device__ __forceinline__ float max128(const float (&v)[128]) {
-  float a[43], b[15], c[5];
-#pragma unroll
-  for (int i = 0; i < 42; ++i) a[i] = fmax3(v[3 * i], v[3 * i + 1], v[3 * i + 2]);
-  a[42] = fmaxf(v[126], v[127]);
-#pragma unroll
-  for (int i = 0; i < 14; ++i) b[i] = fmax3(a[3 * i], a[3 * i + 1], a[3 * i + 2]);
-  b[14] = a[42];
-#pragma unroll
-  for (int i = 0; i < 5; ++i) c[i] = fmax3(b[3 * i], b[3 * i + 1], b[3 * i + 2]);
-  return fmax3(fmax3(c[0], c[1], c[2]), c[3], c[4]);
-}
-__device__ __forceinline__ float min128(const float (&v)[128]) {
-  float a[43], b[15], c[5];
-#pragma unroll
-  for (int i = 0; i < 42; ++i) a[i] = fmin3(v[3 * i], v[3 * i + 1], v[3 * i + 2]);
-  a[42] = fminf(v[126], v[127]);
-#pragma unroll
-  for (int i = 0; i < 14; ++i) b[i] = fmin3(a[3 * i], a[3 * i + 1], a[3 * i + 2]);
-  b[14] = a[42];
-#pragma unroll
-  for (int i = 0; i < 5; ++i) c[i] = fmin3(b[3 * i], b[3 * i + 1], b[3 * i + 2]);
-  return fmin3(fmin3(c[0], c[1], c[2]), c[3], c[4]);
 }
 
 }  // namespace qbsa
