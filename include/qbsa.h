@@ -225,7 +225,7 @@ qbsa_status qbsa_check(void* stream);
 /* Thread-local description of the last non-OK status returned on this thread. */
 const char* qbsa_last_error(void);
 
-/* Library ABI version (major * 100 + minor). */
+/* Library ABI version (major * 100 + minor): 101 (1.01 added qbsa_block_mean, qbsa_block_topk, qbsa_wait_selftest). */
 int qbsa_version(void);
 
 #ifdef __cplusplus

@@ -123,7 +123,7 @@ qbsa_status launch_dense(qbsa::DenseParams& prm, int64_t n_work, cudaStream_t st
 
 extern "C" {
 
-int qbsa_version(void) { return 100; }
+int qbsa_version(void) { return 101; }
 
 const char* qbsa_last_error(void) { return g_last_error.c_str(); }
 
