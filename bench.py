@@ -36,8 +36,8 @@ FP8_OVER_BF16 = 2.0  # nominal dense ratio (4.5 vs 2.25 PFLOP/s), applied to the
 # one ncu capture at S=16384, keep 0.1 (profiles/attn_qbsa_kernel_S16384_keep0.1_full.md); it holds
 # only for the kernel sources it was taken on, identified by their sha1.
 QBSA_NCU_TRAFFIC = {"sources": {"quantized_block_sparse_attn_b200/csrc/attn_qbsa.cuh": "0c45e37fece52e451172bdc93f6c1a699b3ac111",
-                                "quantized_block_sparse_attn_b200/csrc/ptx_sm100.cuh": "00d0c231a8a4e58beb908f6eea8d5d7d9e7323ad"},
-                    "seq": 16384, "keep": 0.1, "bytes": 459670272, "alg_bytes": 420147200}
+                                "quantized_block_sparse_attn_b200/csrc/ptx_sm100.cuh": "ba4e9cf4f466dda99f2eeba00c5ea92d81618f16"},
+                    "seq": 16384, "keep": 0.1, "bytes": 460022528, "alg_bytes": 420147200}
 
 
 def qbsa_traffic(seq: int, keep: float, alg_bytes: int):
