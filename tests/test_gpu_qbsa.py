@@ -208,6 +208,9 @@ def _qbsa_workload(S, keep, heads_for_oracle, n_qblocks):
         compare_out(got[:, h:h + 1], ref, QUANT_MAX_ABS)
         compare_stats(gmax[:, h:h + 1], gsum[:, h:h + 1], rmax, rsum)
         # reported, not gated: error against the unquantised attention over the same kept blocks
+        # (its element mask is S x S bytes, so only up to S = 64K)
+        if S > 65536:
+            continue
         rows = np.concatenate([np.arange(b_ * 128, b_ * 128 + 128) for b_ in qbs])
         keep_el = np.repeat(np.repeat(bm[0, h], 128, axis=0), 128, axis=1)
         dref, _, _ = dense.attention_forward(q[sl], k[sl], v[sl], layout="BNSD", scale=c["scale"],
@@ -224,3 +227,9 @@ def test_qbsa_workload_8k_sampled(keep):
 @pytest.mark.slow
 def test_qbsa_workload_64k_sampled():
     _qbsa_workload(65536, 0.1, heads_for_oracle=[0, 21], n_qblocks=4)
+
+
+@pytest.mark.slow
+def test_qbsa_workload_128k_keep_half_sampled():
+    """The largest configuration of the workload: S = 128K, half the blocks kept."""
+    _qbsa_workload(131072, 0.5, heads_for_oracle=[7], n_qblocks=2)
