@@ -72,9 +72,9 @@ def test_qbsa_unequal_tile_pairs(sign):
 
 
 @pytest.mark.parametrize("sign", [1.0, -1.0])
-def test_qbsa_many_units_per_cta(sign):
-    """More query-block pairs than SMs, so every CTA of the persistent grid walks several
-    (head, pair) units back to back: ragged lengths, GQA, empty and unequal mask rows."""
+def test_qbsa_more_units_than_sms(sign):
+    """More (head, query-block pair) units than SMs, so the grid runs in several waves and
+    CTAs start while others finish: ragged lengths, GQA, empty and unequal mask rows."""
     B, Nq, Nkv, Sq, Skv, D = 2, 40, 8, 1000, 777, 128
     nqb, nkb = 8, 7
     q = iid_normal_bf16(24, 0, B, Nq, Sq, D)
