@@ -163,15 +163,6 @@ __device__ __forceinline__ int compact_mask_row_v16(const uint8_t* row, int n_kb
   return count;
 }
 
-// Lane 0 waits for the phase; the warp synchronises on it (callers then fence with
-// tcgen05.fence::after_thread_sync before touching TMEM).
-__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
-  int ok = 1;
-  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort_flag) ? 1 : 0;
-  __syncwarp();
-  return __shfl_sync(0xffffffffu, ok, 0) != 0;
-}
-
 __global__ void __launch_bounds__(352, 1) attn_qbsa_kernel(const __grid_constant__ QbsaParams p) {
   using C = QbsaCfg;
   extern __shared__ uint8_t smem_raw[];

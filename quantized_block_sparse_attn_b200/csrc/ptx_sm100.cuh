@@ -84,6 +84,15 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   }
 }
 
+// Lane 0 waits for the phase; the warp synchronises on it (callers then fence with
+// tcgen05.fence::after_thread_sync before touching TMEM).
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+  int ok = 1;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort_flag) ? 1 : 0;
+  __syncwarp();
+  return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
 // Cleanup wait: bounded by the same time limit but not by the abort flag, so a CTA that
 // aborted can still let its own asynchronous copies and MMAs land before it exits.
 __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
@@ -314,6 +323,18 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       : "memory");
 }
 
+// Store 64 consecutive 32-bit columns (issue only; pair with tmem_st_wait).
+__device__ __forceinline__ void tmem_st64(uint32_t taddr, const uint32_t (&r)[64]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x64.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,"
+      "%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,"
+      "%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63,%64};" ::"r"(taddr),
+      QBSA_W8(0), QBSA_W8(8), QBSA_W8(16), QBSA_W8(24), QBSA_W8(32), QBSA_W8(40), QBSA_W8(48), QBSA_W8(56)
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_st1(uint32_t taddr, uint32_t v) {
   asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(v) : "memory");
 }
@@ -366,7 +387,17 @@ __device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
   return r;
 }
 
-// As fma_exp2_e4m3x4, from four s32 scores (exact in f32: |s| < 2^24).
+// d = a * b + c for two lanes at once (fma.rn.f32x2, each lane rounded as fmaf); b and c
+// are packed pairs.
+__device__ __forceinline__ void fma_f32x2(float a0, float a1, uint64_t b, uint64_t c, float& d0, float& d1) {
+  asm("{\n\t.reg .b64 a, d;\n\tmov.b64 a, {%2, %3};\n\tfma.rn.f32x2 d, a, %4, %5;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "l"(b), "l"(c));
+}
+
+// Four FP8 weights from four s32 scores (exact in f32: |s| < 2^24): z = s * c + nr on
+// packed pairs (cc, nr hold c and -R twice), p = 2^z (ex2.approx), rounded to FP16 and
+// then to E4M3 (both nearest even, E4M3 saturating); byte i of the result is weight i.
 __device__ __forceinline__ uint32_t i2f_fma_exp2_e4m3x4(uint32_t s0, uint32_t s1, uint32_t s2, uint32_t s3,
                                                         uint64_t cc, uint64_t nr) {
   uint32_t r;

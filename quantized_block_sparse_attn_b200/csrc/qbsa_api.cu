@@ -14,6 +14,7 @@
 
 #include "../../include/qbsa.h"
 #include "attn_dense.cuh"
+#include "attn_pair.cuh"
 #include "attn_qbsa.cuh"
 #include "estimate.cuh"
 #include "quantize.cuh"
@@ -287,11 +288,42 @@ static qbsa_status attn_fwd_impl(const void* q, const void* k, const void* v, in
   if ((st = make_map(&prm.tm_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, k, kd, ks, 64)) != QBSA_OK) return st;
   if ((st = make_map(&prm.tm_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, v, kd, ks, 64)) != QBSA_OK) return st;
 
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // unmasked D = 128 BNSD / BSND (no atten_mask, pse or block mask; a band that covers
+  // every (i, j)): two query tiles per CTA sharing each K/V tile
+  const bool pair_path = D == 128 && !tnd && !atten_mask && !pse && !block_mask && sparse_mode == 0 &&
+                         pre >= (int64_t)Sq - 1 && nxt >= (int64_t)Skv - 1;
+  if (pair_path) {
+    qbsa::PairParams pp;
+    memset(&pp, 0, sizeof(pp));
+    pp.tm_q = prm.tm_q;
+    pp.tm_k = prm.tm_k;
+    pp.tm_v = prm.tm_v;
+    if ((st = make_map(&pp.tm_o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, attention_out, qd, qs, 64)) != QBSA_OK) return st;
+    pp.softmax_max = softmax_max;
+    pp.softmax_sum = softmax_sum;
+    pp.B = B;
+    pp.Nq = Nq;
+    pp.Nkv = Nkv;
+    pp.Sq = Sq;
+    pp.Skv = Skv;
+    pp.group = Nq / Nkv;
+    pp.n_qtiles = (Sq + qbsa::kTile - 1) / qbsa::kTile;
+    pp.n_ktiles = (Skv + qbsa::kTile - 1) / qbsa::kTile;
+    pp.n_pair = (pp.n_qtiles + 1) / 2;
+    pp.n_rank = B * pp.n_pair;
+    pp.head_grp = prm.head_grp;
+    pp.scale = scale;
+    const int64_t n_pw = (int64_t)pp.n_rank * Nq;
+    if ((st = set_smem(qbsa::attn_pair_kernel, qbsa::PairCfg::kSmemBytes)) != QBSA_OK) return st;
+    qbsa::attn_pair_kernel<<<dim3(static_cast<unsigned>(n_pw)), qbsa::PairCfg::kThreads, qbsa::PairCfg::kSmemBytes,
+                             s>>>(pp);
+    return check_launch("attn_pair_kernel launch");
+  }
   if (block_mask) {
     prm.block_mask = block_mask;
     prm.mask_nkb = (Skv + qbsa::kTile - 1) / qbsa::kTile;
   }
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   return D == 128 ? launch_dense<128>(prm, n_work, s) : launch_dense<64>(prm, n_work, s);
 }
 

@@ -47,6 +47,9 @@ def _run_and_compare(q, k, v, layout, Nq, scale, mode=0, pre=INF, nxt=INF, mask=
     (2, 2, 1, 520, 520, 64, 0, 100, 20, "BSND"),       # band
     (1, 1, 1, 640, 640, 128, 0, -50, 200, "BNSD"),     # band excluding the diagonal
     (1, 1, 1, 1, 1, 128, 0, INF, INF, "BNSD"),
+    # unmasked D = 128 (two query tiles per CTA): BSND, an odd tile count, one short K tile
+    (1, 3, 1, 650, 333, 128, 0, INF, INF, "BSND"),
+    (2, 2, 2, 129, 100, 128, 0, INF, INF, "BNSD"),
     (1, 1, 1, 1, 700, 64, 3, INF, INF, "BNSD"),
     (1, 3, 1, 1000, 1000, 128, 2, INF, INF, "BNSD"),
 ])
@@ -94,7 +97,7 @@ def test_dense_tnd_gqa_causal(D):
 
 
 @pytest.mark.parametrize("mode,pre,nxt,layout", [(0, 300, 40, "BNSD"), (2, INF, INF, "BNSD"), (3, INF, INF, "BSND"),
-                                                 (3, INF, INF, "TND")])
+                                                 (3, INF, INF, "TND"), (0, INF, INF, "BNSD"), (0, INF, INF, "BSND")])
 def test_mask_logic_bit_exact_via_zero_query(mode, pre, nxt, layout):
     """Q = 0 makes every kept weight exactly 1: softmax_sum must equal the kept-key count."""
     D, Nq, Nkv = 128, 2, 1
