@@ -35,9 +35,9 @@ FP8_OVER_BF16 = 2.0  # nominal dense ratio (4.5 vs 2.25 PFLOP/s), applied to the
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one attn_qbsa_kernel launch from
 # one ncu capture at S=16384, keep 0.1 (profiles/attn_qbsa_kernel_S16384_keep0.1_full.md); it holds
 # only for the kernel sources it was taken on, identified by their sha1.
-QBSA_NCU_TRAFFIC = {"sources": {"quantized_block_sparse_attn_b200/csrc/attn_qbsa.cuh": "0c45e37fece52e451172bdc93f6c1a699b3ac111",
-                                "quantized_block_sparse_attn_b200/csrc/ptx_sm100.cuh": "ba4e9cf4f466dda99f2eeba00c5ea92d81618f16"},
-                    "seq": 16384, "keep": 0.1, "bytes": 460022528, "alg_bytes": 420147200}
+QBSA_NCU_TRAFFIC = {"sources": {"quantized_block_sparse_attn_b200/csrc/attn_qbsa.cuh": "5a21fd90ccb9d35f74b4398bc7764686c1cf59fe",
+                                "quantized_block_sparse_attn_b200/csrc/ptx_sm100.cuh": "76287e5abe014dfeeab1944e7be8a2564b0e0057"},
+                    "seq": 16384, "keep": 0.1, "bytes": 456649216, "alg_bytes": 420147200}
 
 
 def qbsa_traffic(seq: int, keep: float, alg_bytes: int):
@@ -523,7 +523,7 @@ def dense_line(device, stream, S, warmup, steps, bf16_peak, dist):
     del q, k, v, out
     torch.cuda.empty_cache()
     return {"workload": f"attn_fwd bf16 B=1 N=40 S={S} D=128 no mask", "ms": ms, "tflops": flops / ms / 1e9,
-            "pct_of_bf16_peak": 100 * flops / ms / 1e9 / bf16_peak, "kernel": "attn_dense_kernel<128>"}
+            "pct_of_bf16_peak": 100 * flops / ms / 1e9 / bf16_peak, "kernel": "attn_pair_kernel"}
 
 
 def main():
