@@ -86,6 +86,17 @@ static_assert(PairCfg::kSmemBytes <= 232448, "shared memory above the 227 KB opt
 static_assert(PairCfg::kKOff % 1024 == 0 && PairCfg::kVOff % 1024 == 0 && PairCfg::kTileBytes % 1024 == 0,
               "swizzled buffers must start on 1024-byte boundaries");
 
+// acc += (a, b) on two packed f32 lanes (add.rn.f32x2: one instruction per pair of scores).
+__device__ __forceinline__ void add_f32x2(uint64_t& acc, float a, float b) {
+  asm("{\n\t.reg .b64 q;\n\tmov.b64 q, {%1, %2};\n\tadd.rn.f32x2 %0, %0, q;\n\t}" : "+l"(acc) : "f"(a), "f"(b));
+}
+// Sum of the two f32 lanes of a packed pair.
+__device__ __forceinline__ float sum_f32x2(uint64_t v) {
+  float a, b;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+  return a + b;
+}
+
 __global__ void __launch_bounds__(352, 1) attn_pair_kernel(const __grid_constant__ PairParams p) {
   using C = PairCfg;
   extern __shared__ uint8_t smem_raw[];
@@ -328,17 +339,17 @@ __global__ void __launch_bounds__(352, 1) attn_pair_kernel(const __grid_constant
       const uint64_t cc = pack_f32x2(c, c);
       const uint64_t nm = pack_f32x2(-mc, -mc);
       uint32_t pk[64];
-      float ls[4] = {0.f, 0.f, 0.f, 0.f};  // independent partial sums (short dependency chains)
+      uint64_t acc[2] = {0ull, 0ull};  // packed partial row sums: two pairs of lanes
 #pragma unroll
       for (int x = 0; x < 64; ++x) {
         float z0, z1;
         fma_f32x2(sv[2 * x], sv[2 * x + 1], cc, nm, z0, z1);
         const float p0 = ex2(z0);
         const float p1 = ex2(z1);
-        ls[x & 3] += p0 + p1;
+        add_f32x2(acc[x & 1], p0, p1);
         pk[x] = pack_bf16x2(p0, p1);
       }
-      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      l += sum_f32x2(acc[0]) + sum_f32x2(acc[1]);
 
       // P_t and O_t are free once the previous block's P·V has retired
       if (j > 0) {
