@@ -5,7 +5,9 @@
 // CTA, streaming 128-row K/V tiles with an online softmax so that the score matrix
 // never reaches global memory (§2, the tiling remark).  Masks follow §4.2/§4.3,
 // varlen TND follows §4.3, GQA follows §7, and the outputs are attention_out,
-// softmax_max and softmax_sum (§5).
+// softmax_max and softmax_sum (§5).  The unmasked D = 128 BNSD / BSND case goes to
+// attn_pair_kernel (two query tiles per CTA, attn_pair.cuh); this kernel serves every
+// other case, including bsa_fwd's block lists.
 //
 // CTA = 10 warps:
 //   warp 0      TMA producer: Q once, then K/V tiles into a 2-stage ring each.
