@@ -164,7 +164,7 @@ def test_video_workload_sampled():
 
 
 @pytest.mark.parametrize("B,Nq,Nkv,S,D,keep", [(1, 2, 1, 300, 128, 0.5), (2, 2, 2, 1024, 64, 0.25),
-                                               (1, 3, 1, 640, 128, 1.0)])
+                                               (1, 3, 1, 640, 128, 1.0), (2, 4, 2, 2048, 128, 0.3)])
 def test_bsa_parity(B, Nq, Nkv, S, D, keep):
     """bf16 block-sparse attention = the dense oracle with the unkept blocks masked."""
     from workloads import block_keep_mask
