@@ -1,5 +1,8 @@
 """Quantized block-sparse attention forward (EagleQBSA), step by step in fp64.
 
+TEST INFRASTRUCTURE ONLY (see the package docstring): nothing in the product path
+imports this module.
+
 Source: EagleQBSA article, "昇腾MindIE SD高性能量化稀疏联合注意力EagleQBSA,视频生成端到端加速1.6倍".
 
 * Section "EagleQBSA量化叠加稀疏方案设计" and Fig 2.1: Q and K are quantised to
@@ -24,35 +27,48 @@ Readings where the article is silent (each also listed in the design notes):
 * Shapes: query_scale [B, N_q, ceil(S_q/128)], key_scale [B, N_kv, ceil(S_kv/128)],
   value_scale [B, N_kv, D]; block_sparse_mask uint8 [B, N_q, ceil(S_q/128),
   ceil(S_kv/128)] with 1 = compute the block.
-* Score: s = t * s_q * s_k * scale, t the exact integer dot product of the INT8 rows;
-  z = s * log2(e) is the same score in base-2 units.
-* Kept blocks are visited in ascending key order, one 128-key block per step.  The
-  weights are taken against a power-of-two reference R (an integer in log2 units)
-  that follows the running max m of z lazily: at a block, m = max(m, rowmax z); if R
-  is unset or m > R + 8, R = ceil(m) and the accumulated l and acc are multiplied by
-  the exact power of two 2^(R_old - R).  Then p = 2^(z - R) <= 2^8 (below E4M3's 448).
-  The article fixes neither the reference nor when it moves.  A power-of-two
-  reference makes the rescaling exact, and E4M3 rounding commutes with powers of two,
-  so the codes equal those against the final max except for weights in E4M3's
-  subnormal range (below 2^-6 of the reference).
-* p is held in FP16 before its FP8 rounding, the precision the article gives for P
+* Score: s = t * s_q * s_k * scale, t the exact integer dot product of the INT8 rows.
+* P is held in FP16 before its FP8 rounding, the precision the article gives for P
   (section "昇腾亲和的量化叠加稀疏Attention算子优化": the FP16 P matrix is converted
-  to FP8): p16 = FP16(2^(z - R)) and p8 = E4M3(p16), both nearest even; the FP8
-  decision is taken on p16 on both sides.  l = Σ p8 (the sum of the ROUNDED
-  weights, so constant V returns V exactly); O[:, c] = acc[:, c] / l · v_scale[c]
-  with acc = Σ p8 · v8.
-* softmax_max = final m in the natural-log domain (max s) and softmax_sum = l · 2^(R - m):
-  the sum of the rounded weights expressed against the true row maximum.
+  to FP8): p8 = E4M3(FP16(p)), both nearest even; the FP8 decision is taken on the
+  FP16 value on both sides.
+* l = Σ p8, the sum of the ROUNDED weights (so constant V returns V exactly);
+  O[:, c] = acc[:, c] / l · v_scale[c] with acc = Σ p8 · v8.
 * A row with no kept block returns O = 0, softmax_max = -inf, softmax_sum = 0.
+
+Which maximum p is taken against decides the FP8 codes, and the article does not say.
+Two readings are written out here:
+
+* ``qbsa_forward`` -- the plain online-softmax definition.  Kept blocks are visited
+  in ascending key order, one 128-key block per step; the running max m (natural-log
+  units) moves at every block, m_new = max(m, rowmax s); the accumulated l and acc
+  are multiplied by e^(m - m_new) at every step; the block's weights are
+  p8 = E4M3(FP16(e^(s - m_new))).  softmax_max = final m, softmax_sum = final l.
+  No choice made for a kernel's speed enters it.
+* ``qbsa_forward_pow2ref`` -- the reading the CUDA kernel takes.  The same visit
+  order, but the weights are taken against a power-of-two reference R (an integer in
+  log2 units, z = s · log2 e) that follows the running max lazily: at a block,
+  m = max(m, rowmax z); if R is unset or m > R + 8, R = ceil(m) and l, acc are
+  multiplied by the exact power of two 2^(R_old - R).  Then p8 = E4M3(FP16(2^(z - R)))
+  with 2^(z - R) <= 2^8 (below E4M3's 448).  softmax_sum = l · 2^(R - m): the rounded
+  weights' sum against the true row maximum.  Because R is a power of two, E4M3
+  rounding commutes with every rescale, so the codes equal those against the last
+  reference except for weights in E4M3's subnormal range; against the plain reading
+  they differ by one rounding of each weight on a shifted grid, well inside the
+  quantized tolerance.
 
 Parity pins (tests): the quantiser codes meet the rounding bound |x - q s| <= s/2 and
 hit ±127 at the block maximum; the E4M3 codec matches the OCP definition on every
-code and torch's float8_e4m3fn cast on finite inputs; with P rounding switched off the
-result equals the dense oracle restricted to the kept blocks; q = 0 gives p8 = 1,
-softmax_sum = the kept-key count and O = the mean of the dequantised V; constant V
-returns V; a pure-Python loop version agrees on tiny inputs; masked-out blocks have no
-influence.  The article prints no quantisation error figure ("parity unpinned" for
-the article's own error level; only VBench scores are given, out of scope).
+code and torch's float8_e4m3fn cast on finite inputs, and the FP16 -> E4M3 double
+rounding matches torch's float16 -> float8_e4m3fn casts on a dense grid; for both
+readings, with P rounding switched off the result equals the direct softmax over the
+kept blocks, q = 0 gives p8 = 1, softmax_sum = the kept-key count and O = the mean of
+the dequantised V, constant V returns V, a pure-Python loop version agrees on tiny
+inputs, and masked-out blocks have no influence; the plain reading with a single kept
+block per row equals the closed form E4M3(FP16(e^(s - max s))), and both readings lie
+within the per-weight E4M3 bound of the unrounded softmax.  The article prints no
+quantisation error figure ("parity unpinned" for the article's own error level; only
+VBench scores are given, out of scope).
 """
 
 from __future__ import annotations
@@ -65,7 +81,7 @@ from .formats import bf16_to_f64, e4m3_encode, e4m3_decode
 
 BLK = 128
 LOG2E = 1.0 / math.log(2.0)
-REF_SLACK = 8  # the reference is re-set once the running max exceeds it by more than 8 (log2 units)
+REF_SLACK = 8  # pow2 reading: the reference is re-set once the running max exceeds it by more than 8 (log2 units)
 
 
 # --------------------------------------------------------------------------------------
@@ -110,22 +126,63 @@ def quantize_v_per_channel(v):
 # the forward
 # --------------------------------------------------------------------------------------
 
-def _head_forward(q8, k8, qs, ks, v8f, vs, mask_rows, scale, qbs, round_p=True):
-    """One (b, h): q8 [Sq, D] int8, k8 [Skv, D], v8f [Skv, D] decoded E4M3, per-block scales."""
+def _fp8_weights(p):
+    """p (fp64, >= 0) -> E4M3(FP16(p)) as fp64: the weight held in FP16, then rounded to FP8."""
+    return e4m3_decode(e4m3_encode(p.astype(np.float16).astype(np.float32)))
+
+
+def _block_scores(qi, k8, qs_b, ks_b, scale, c0, c1):
+    """s = t · s_q · s_k · scale for one kept key block, t the exact integer dot products."""
+    t = qi @ k8[c0:c1].astype(np.int64).T
+    return t.astype(np.float64) * (float(qs_b) * float(ks_b) * scale)
+
+
+def _head_plain(q8, k8, qs, ks, v8f, vs, mask_rows, scale, qbs, round_p=True):
+    """Plain online-softmax reading for one (b, h): running max moved and l, acc rescaled
+    at every kept block; weights E4M3(FP16(e^(s - m))) against that running max."""
     skv, D = k8.shape[0], v8f.shape[1]
     outs, mxs, sms = [], [], []
     for qb in qbs:
         r0, r1 = qb * BLK, min(q8.shape[0], (qb + 1) * BLK)
         rows = r1 - r0
         qi = q8[r0:r1].astype(np.int64)
-        m = np.full(rows, -np.inf)     # running max of z
+        m = np.full(rows, -np.inf)     # running max of s (natural-log units)
+        l = np.zeros(rows)
+        acc = np.zeros((rows, D))
+        for kb in np.nonzero(mask_rows[qb])[0]:                               # ascending
+            c0, c1 = kb * BLK, min(skv, (kb + 1) * BLK)
+            s = _block_scores(qi, k8, qs[qb], ks[kb], scale, c0, c1)
+            m_new = np.maximum(m, s.max(axis=1))
+            alpha = np.exp(m - m_new)                                          # 0 while m = -inf
+            p = np.exp(s - m_new[:, None])
+            if round_p:
+                p = _fp8_weights(p)
+            l = l * alpha + p.sum(axis=1)
+            acc = acc * alpha[:, None] + p @ v8f[c0:c1]
+            m = m_new
+        live = l > 0
+        outs.append(np.where(live[:, None], acc / np.where(live, l, 1.0)[:, None], 0.0) * vs[None, :])
+        mxs.append(m)
+        sms.append(np.where(live, l, 0.0))
+    return outs, mxs, sms
+
+
+def _head_pow2ref(q8, k8, qs, ks, v8f, vs, mask_rows, scale, qbs, round_p=True):
+    """Kernel's reading for one (b, h): weights E4M3(FP16(2^(z - R))) against a lazily moved
+    power-of-two reference R (re-set to ceil(m) only when m passes R + REF_SLACK)."""
+    skv, D = k8.shape[0], v8f.shape[1]
+    outs, mxs, sms = [], [], []
+    for qb in qbs:
+        r0, r1 = qb * BLK, min(q8.shape[0], (qb + 1) * BLK)
+        rows = r1 - r0
+        qi = q8[r0:r1].astype(np.int64)
+        m = np.full(rows, -np.inf)     # running max of z (log2 units)
         ref = np.full(rows, -np.inf)   # power-of-two reference R (an integer)
         l = np.zeros(rows)
         acc = np.zeros((rows, D))
         for kb in np.nonzero(mask_rows[qb])[0]:                               # ascending
             c0, c1 = kb * BLK, min(skv, (kb + 1) * BLK)
-            t = qi @ k8[c0:c1].astype(np.int64).T                              # exact integers
-            z = t.astype(np.float64) * (float(qs[qb]) * float(ks[kb]) * scale) * LOG2E
+            z = _block_scores(qi, k8, qs[qb], ks[kb], scale, c0, c1) * LOG2E
             m = np.maximum(m, z.max(axis=1))
             upd = np.isneginf(ref) | (m > ref + REF_SLACK)
             new_ref = np.where(upd, np.ceil(m), ref)
@@ -134,7 +191,7 @@ def _head_forward(q8, k8, qs, ks, v8f, vs, mask_rows, scale, qbs, round_p=True):
             l, acc, ref = l * alpha, acc * alpha[:, None], new_ref
             p = np.exp2(z - ref[:, None])
             if round_p:
-                p = e4m3_decode(e4m3_encode(p.astype(np.float16).astype(np.float32)))
+                p = _fp8_weights(p)
             l = l + p.sum(axis=1)
             acc = acc + p @ v8f[c0:c1]
         live = l > 0
@@ -144,18 +201,7 @@ def _head_forward(q8, k8, qs, ks, v8f, vs, mask_rows, scale, qbs, round_p=True):
     return outs, mxs, sms
 
 
-def qbsa_forward(q8, k8, q_scale, k_scale, v8, v_scale, block_mask, scale: float,
-                 heads=None, q_blocks=None, round_p: bool = True):
-    """Oracle of the quantized block-sparse forward (BNSD).
-
-    q8 [B, Nq, Sq, D] int8; k8 [B, Nkv, Skv, D] int8; q_scale [B, Nq, ceil(Sq/128)];
-    k_scale [B, Nkv, ceil(Skv/128)]; v8 [B, Nkv, Skv, D] E4M3 codes (uint8);
-    v_scale [B, Nkv, D]; block_mask [B, Nq, ceil(Sq/128), ceil(Skv/128)] uint8, 1 = compute.
-
-    Returns (out [B, Nq, Sq, D], softmax_max [B, Nq, Sq], softmax_sum [B, Nq, Sq]) in
-    fp64.  ``heads`` / ``q_blocks`` restrict the work for sampled checks (other entries
-    NaN).  ``round_p=False`` skips the FP8 rounding of P (used only by a pin).
-    """
+def _forward(head_fn, q8, k8, q_scale, k_scale, v8, v_scale, block_mask, scale, heads, q_blocks, round_p):
     q8 = np.asarray(q8)
     k8 = np.asarray(k8)
     B, Nq, Sq, D = q8.shape
@@ -172,9 +218,8 @@ def qbsa_forward(q8, k8, q_scale, k_scale, v8, v_scale, block_mask, scale: float
         g = h // group
         if (b, g) not in v8f_cache:
             v8f_cache[(b, g)] = e4m3_decode(v8[b, g])
-        o, mx, sm = _head_forward(q8[b, h], k8[b, g], q_scale[b, h], k_scale[b, g], v8f_cache[(b, g)],
-                                  np.asarray(v_scale[b, g], dtype=np.float64), block_mask[b, h], scale, qbs,
-                                  round_p)
+        o, mx, sm = head_fn(q8[b, h], k8[b, g], q_scale[b, h], k_scale[b, g], v8f_cache[(b, g)],
+                            np.asarray(v_scale[b, g], dtype=np.float64), block_mask[b, h], scale, qbs, round_p)
         for qb, oo, mm, ss in zip(qbs, o, mx, sm):
             r0, r1 = qb * BLK, min(Sq, (qb + 1) * BLK)
             out[b, h, r0:r1] = oo
@@ -183,8 +228,31 @@ def qbsa_forward(q8, k8, q_scale, k_scale, v8, v_scale, block_mask, scale: float
     return out, smax, ssum
 
 
-def qbsa_forward_loops(q8, k8, q_scale, k_scale, v8, v_scale, block_mask, scale: float):
-    """The same forward with explicit Python loops over rows and keys (tiny inputs)."""
+def qbsa_forward(q8, k8, q_scale, k_scale, v8, v_scale, block_mask, scale: float,
+                 heads=None, q_blocks=None, round_p: bool = True):
+    """Oracle of the quantized block-sparse forward (BNSD), plain online-softmax reading.
+
+    q8 [B, Nq, Sq, D] int8; k8 [B, Nkv, Skv, D] int8; q_scale [B, Nq, ceil(Sq/128)];
+    k_scale [B, Nkv, ceil(Skv/128)]; v8 [B, Nkv, Skv, D] E4M3 codes (uint8);
+    v_scale [B, Nkv, D]; block_mask [B, Nq, ceil(Sq/128), ceil(Skv/128)] uint8, 1 = compute.
+
+    Returns (out [B, Nq, Sq, D], softmax_max [B, Nq, Sq], softmax_sum [B, Nq, Sq]) in
+    fp64.  ``heads`` / ``q_blocks`` restrict the work for sampled checks (other entries
+    NaN).  ``round_p=False`` skips the FP8 rounding of P (used only by a pin).
+    """
+    return _forward(_head_plain, q8, k8, q_scale, k_scale, v8, v_scale, block_mask, scale, heads, q_blocks,
+                    round_p)
+
+
+def qbsa_forward_pow2ref(q8, k8, q_scale, k_scale, v8, v_scale, block_mask, scale: float,
+                         heads=None, q_blocks=None, round_p: bool = True):
+    """The same forward with the weights taken against the lazily moved power-of-two
+    reference (the CUDA kernel's reading; module docstring).  Same arguments and returns."""
+    return _forward(_head_pow2ref, q8, k8, q_scale, k_scale, v8, v_scale, block_mask, scale, heads, q_blocks,
+                    round_p)
+
+
+def _loops(q8, k8, q_scale, k_scale, v8, v_scale, block_mask, scale, pow2ref):
     q8 = np.asarray(q8)
     k8 = np.asarray(k8)
     B, Nq, Sq, D = q8.shape
@@ -204,19 +272,29 @@ def qbsa_forward_loops(q8, k8, q_scale, k_scale, v8, v_scale, block_mask, scale:
                     if not block_mask[b, h, qb, kb]:
                         continue
                     cols = range(kb * BLK, min(Skv, (kb + 1) * BLK))
-                    z = []
+                    s = []
                     for j in cols:
                         t = sum(int(q8[b, h, i, c]) * int(k8[b, g, j, c]) for c in range(D))
-                        z.append(t * (float(q_scale[b, h, qb]) * float(k_scale[b, g, kb]) * scale) * LOG2E)
-                    m = max(m, max(z))
-                    if ref == -math.inf or m > ref + REF_SLACK:
-                        new_ref = math.ceil(m)
-                        alpha = 0.0 if ref == -math.inf else 2.0 ** (ref - new_ref)
+                        s.append(t * (float(q_scale[b, h, qb]) * float(k_scale[b, g, kb]) * scale))
+                    if pow2ref:
+                        z = [x * LOG2E for x in s]
+                        m = max(m, max(z))
+                        if ref == -math.inf or m > ref + REF_SLACK:
+                            new_ref = math.ceil(m)
+                            alpha = 0.0 if ref == -math.inf else 2.0 ** (ref - new_ref)
+                            l *= alpha
+                            acc = [a * alpha for a in acc]
+                            ref = new_ref
+                        ws = [2.0 ** (zj - ref) for zj in z]
+                    else:
+                        m_new = max(m, max(s))
+                        alpha = 0.0 if m == -math.inf else math.exp(m - m_new)
                         l *= alpha
                         acc = [a * alpha for a in acc]
-                        ref = new_ref
-                    for j, zj in zip(cols, z):
-                        p16 = np.float16(2.0 ** (zj - ref))           # P held in FP16 first
+                        m = m_new
+                        ws = [math.exp(sj - m) for sj in s]
+                    for j, w in zip(cols, ws):
+                        p16 = np.float16(w)                                   # P held in FP16 first
                         p = float(e4m3_decode(e4m3_encode(np.float32(p16))))
                         l += p
                         vrow = e4m3_decode(v8[b, g, j])
@@ -225,6 +303,93 @@ def qbsa_forward_loops(q8, k8, q_scale, k_scale, v8, v_scale, block_mask, scale:
                 if l > 0:
                     for c in range(D):
                         out[b, h, i, c] = acc[c] / l * float(v_scale[b, g, c])
-                    smax[b, h, i] = m / LOG2E
-                    ssum[b, h, i] = l * 2.0 ** (ref - m)
+                    if pow2ref:
+                        smax[b, h, i] = m / LOG2E
+                        ssum[b, h, i] = l * 2.0 ** (ref - m)
+                    else:
+                        smax[b, h, i] = m
+                        ssum[b, h, i] = l
     return out, smax, ssum
+
+
+def qbsa_forward_loops(q8, k8, q_scale, k_scale, v8, v_scale, block_mask, scale: float):
+    """``qbsa_forward`` with explicit Python loops over rows and keys (tiny inputs)."""
+    return _loops(q8, k8, q_scale, k_scale, v8, v_scale, block_mask, scale, pow2ref=False)
+
+
+def qbsa_forward_pow2ref_loops(q8, k8, q_scale, k_scale, v8, v_scale, block_mask, scale: float):
+    """``qbsa_forward_pow2ref`` with explicit Python loops over rows and keys (tiny inputs)."""
+    return _loops(q8, k8, q_scale, k_scale, v8, v_scale, block_mask, scale, pow2ref=True)
+
+
+# --------------------------------------------------------------------------------------
+# how far the power-of-two reading may lie from the plain one
+# --------------------------------------------------------------------------------------
+
+# Relative error of one weight held in FP16 and then rounded to E4M3 in E4M3's normal
+# range: half the E4M3 spacing, 2^-4, plus the FP16 step (2^-11 of the value) and slack
+# for ex2.approx and the fp32 score arithmetic of a kernel.
+P_ROUND_EPS = 2.0 ** -4 + 2.0 ** -10
+
+
+def pow2ref_weight_error(w):
+    """Largest |a - w| for one weight of the power-of-two reading, in units of the row max.
+
+    w = e^(s - max s) is the exact weight.  The reading rounds x = w · 2^(m - R) with the
+    row's log2 max m and R - m in [-8, 1) (R = ceil of a running max, moved once m passes
+    R + 8), so x >= w / 2 and the error in row-max units is 2^(R - m) <= 2 times the error
+    in reference units.  At x >= 2^-6 (E4M3 normal) that error is at most P_ROUND_EPS · x;
+    below, the E4M3 spacing is 2^-9, so it is at most min(x, 2^-10) (a value under 2^-10
+    rounds to 0) plus the FP16 step.  Hence e(w) = P_ROUND_EPS·w + [w < 2^-5]·min(w, 2^-9),
+    with a 1e-3 margin on the threshold and the clamp, and 2^-24 for FP16's subnormal step.
+    """
+    w = np.asarray(w, dtype=np.float64)
+    sub = np.where(w < 2.0 ** -5 * 1.001, np.minimum(1.001 * w, 2.0 ** -9), 0.0)
+    return P_ROUND_EPS * w + sub + 2.0 ** -24
+
+
+def qbsa_reading_gap_terms(q8, k8, q_scale, k_scale, v8, v_scale, block_mask, scale: float, center,
+                           heads=None, q_blocks=None):
+    """Terms of the bound on |O_a - O_p| between any output O_a whose weights a_i lie within
+    pow2ref_weight_error(w_i) of the exact weights and the plain reading's output O_p.
+
+    With A = Σ a_i, W = Σ w_i and O_w the unrounded output (qbsa_forward with round_p=False):
+        O_a - O_p = [Σ_i (a_i - w_i)(v_i - O_p) + W (O_w - O_p)] / A,
+    since Σ_i a_i (v_i - O_p) = A (O_a - O_p) and Σ_i w_i (v_i - O_p) = W (O_w - O_p).  So
+        |O_a - O_p| <= [G + W |O_w - O_p|] / A,   G[c] = Σ_i e(w_i) |v_ic - O_p[c]|,
+    and, for the row sums, |A - l_p| <= E + |W - l_p| with E = Σ_i e(w_i).
+
+    ``center`` is O_p (the plain reading's output, [B, Nq, Sq, D]); v_ic is the dequantised
+    value e4m3(v8)·v_scale.  Returns (G [B, Nq, Sq, D], E [B, Nq, Sq]) over the rows that
+    ``heads`` / ``q_blocks`` select (NaN elsewhere); rows with no kept key get 0.
+    """
+    q8 = np.asarray(q8)
+    k8 = np.asarray(k8)
+    B, Nq, Sq, D = q8.shape
+    Nkv, Skv = k8.shape[1], k8.shape[2]
+    group = Nq // Nkv
+    nqb = -(-Sq // BLK)
+    G = np.full((B, Nq, Sq, D), np.nan)
+    E = np.full((B, Nq, Sq), np.nan)
+    sel = heads if heads is not None else [(b, h) for b in range(B) for h in range(Nq)]
+    qbs = list(range(nqb)) if q_blocks is None else list(q_blocks)
+    for b, h in sel:
+        g = h // group
+        vdq = e4m3_decode(v8[b, g]) * np.asarray(v_scale[b, g], dtype=np.float64)[None, :]
+        for qb in qbs:
+            r0, r1 = qb * BLK, min(Sq, (qb + 1) * BLK)
+            kept = np.nonzero(block_mask[b, h, qb])[0]
+            if len(kept) == 0:
+                G[b, h, r0:r1] = 0.0
+                E[b, h, r0:r1] = 0.0
+                continue
+            qi = q8[b, h, r0:r1].astype(np.int64)
+            s = np.concatenate([_block_scores(qi, k8[b, g], q_scale[b, h, qb], k_scale[b, g, kb], scale,
+                                              kb * BLK, min(Skv, (kb + 1) * BLK)) for kb in kept], axis=1)
+            cols = np.concatenate([np.arange(kb * BLK, min(Skv, (kb + 1) * BLK)) for kb in kept])
+            e = pow2ref_weight_error(np.exp(s - s.max(axis=1, keepdims=True)))
+            E[b, h, r0:r1] = e.sum(axis=1)
+            vk = vdq[cols]
+            for i in range(r1 - r0):
+                G[b, h, r0 + i] = e[i] @ np.abs(vk - center[b, h, r0 + i][None, :])
+    return G, E
