@@ -33,8 +33,8 @@ METRIC = "attention fwd TFLOPS (B=1,N=40,D=128) and % of B200 tensor peak vs S"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FP8_OVER_BF16 = 2.0  # nominal dense ratio (4.5 vs 2.25 PFLOP/s), applied to the measured bf16 peak
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one attn_qbsa_kernel launch from
-# one ncu capture at S=16384, keep 0.1 (profiles/attn_qbsa_kernel_S16384_keep0.1_full.md); it holds
-# only for the kernel sources it was taken on, identified by their sha1.
+# one ncu capture at S=16384, keep 0.1; it holds only for the kernel sources it was taken on,
+# identified by their sha1.
 QBSA_NCU_TRAFFIC = {"sources": {"quantized_block_sparse_attn_b200/csrc/attn_qbsa.cuh": "5a21fd90ccb9d35f74b4398bc7764686c1cf59fe",
                                 "quantized_block_sparse_attn_b200/csrc/ptx_sm100.cuh": "76287e5abe014dfeeab1944e7be8a2564b0e0057"},
                     "seq": 16384, "keep": 0.1, "bytes": 456649216, "alg_bytes": 420147200}
@@ -472,7 +472,7 @@ def estimate_line(device, stream, S, keep, hbm_peak):
     quantized workload's bf16 Q/K recipe at this S."""
     import torch
     import quantized_block_sparse_attn_b200 as qb
-    from workloads import CONFIGS, device_blocky_qk_bf16
+    from workloads import CONFIGS, block_keep_mask, device_blocky_qk_bf16
     c = CONFIGS["qbsa"]
     N, D, seed = c["Nq"], c["D"], c["seed"]
     q = device_blocky_qk_bf16(seed, "q", 1, N, S, D, device)
@@ -493,12 +493,13 @@ def estimate_line(device, stream, S, keep, hbm_peak):
     pool_ms, topk_ms = pool_ms / 5, topk_ms / 5
     pool_bytes = 2 * N * S * D * 2 + 2 * N * nb * D * 4  # bf16 Q and K read, fp32 means written
     kept = int(state["mask"].sum().item())
+    expected = int(block_keep_mask(seed, 1, 1, nb, nb, keep).sum()) * N  # same count rule, one head's rows
     del q, k, state
     torch.cuda.empty_cache()
     return {"workload": f"block-mask estimation B=1 N=40 S={S} D=128 keep={keep}", "ms": pool_ms + topk_ms,
             "block_mean_ms": pool_ms, "block_mean_gbs": pool_bytes / (pool_ms / 1e3) / 1e9,
             "block_mean_frac_of_hbm": pool_bytes / (pool_ms / 1e3) / 1e9 / hbm_peak,
-            "block_topk_ms": topk_ms, "kept_blocks": kept, "expected_kept": N * nb * qb.keep_count(nb, keep),
+            "block_topk_ms": topk_ms, "kept_blocks": kept, "expected_kept": expected,
             "kernels": "block_mean_kernel x2 (HBM-bound), block_topk_kernel"}
 
 

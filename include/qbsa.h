@@ -126,12 +126,21 @@ qbsa_status bsa_fwd(const void* q, const void* k, const void* v, const uint8_t* 
  * block_mask     uint8 [B, Nq, ceil(Sq/128), ceil(Skv/128)], 1 = compute the block
  * D              128 (other values: QBSA_ERR_UNSUPPORTED); ceil(Skv/128) <= 2048.
  * scale          softmax scale (scale_value in [QBSA]'s call, 128^-0.5 there).
- * Score s = int_dot(q_i8, k_i8) * q_scale * k_scale * scale.  Kept key blocks are
- * visited in ascending order and the running max is updated at every block; P is
- * rounded to E4M3 against that running max and the row sum is the sum of the rounded
- * weights.  attention_out bf16 [B, Nq, Sq, D]; softmax_max / softmax_sum optional fp32
- * [B, Nq, Sq] (natural-log max, sum of the rounded weights relative to it).  A row
- * with no kept block gets out = 0, max = -inf, sum = 0.
+ * Score s = int_dot(q_i8, k_i8) * q_scale * k_scale * scale, z = s * log2(e).  Kept
+ * key blocks are visited in ascending order, one 128-key block per step, and the
+ * running max m = max z is updated at every block.  The weights are taken against a
+ * power-of-two reference R (an integer, log2 units): R = ceil(m) at the first kept
+ * block, and again whenever m exceeds R + 8, at which point the accumulated row sum
+ * and output are multiplied by the exact power of two 2^(R_old - R_new).  Each weight
+ * is held in FP16 and then rounded to E4M3: p8 = E4M3(FP16(2^(z - R))), both
+ * round-to-nearest-even, E4M3 saturating ([QBSA] "昇腾亲和的量化叠加稀疏Attention算子优化":
+ * the FP16 P matrix is converted to FP8).  2^(z - R) <= 2^8, below E4M3's 448.  The
+ * row sum L is the sum of the rounded weights; out[:, c] = (Σ p8 v8)[c] / L * v_scale[c].
+ * These codes equal those taken against the plain running max e^(s - m) up to one
+ * E4M3 rounding on a shifted grid.  attention_out bf16 [B, Nq, Sq, D]; softmax_max /
+ * softmax_sum optional fp32 [B, Nq, Sq]: the natural-log row max and L * 2^(R - m),
+ * the rounded weights' sum against that max.  A row with no kept block gets out = 0,
+ * max = -inf, sum = 0.
  */
 qbsa_status qbsa_fwd(const int8_t* q_i8, const int8_t* k_i8, const float* q_block_scale, const float* k_block_scale,
                      const uint8_t* v_fp8, const float* v_channel_scale, const uint8_t* block_mask, int B, int Nq,
@@ -206,6 +215,19 @@ qbsa_status qbsa_block_topk(const float* q_mean, const float* k_mean, int B, int
                             float scale, int n_keep, uint8_t* block_mask, float* block_scores, void* stream);
 
 /*
+ * qbsa_block_topk_keep -- qbsa_block_topk with the count given as a keep fraction: each
+ * query block keeps n_keep = max(1, min(nkb, round(keep * nkb))) key blocks, the product
+ * taken in double and rounded to nearest with ties to even (the count rule of the
+ * keep-10% / keep-50% masks of [QBSA] "EagleQBSA单算子性能验证分析", sparsity 0.9 / 0.5).
+ *   keep        in [0, 1]; other values return QBSA_ERR_INVALID before any launch.
+ *   n_keep_out  host int, or NULL: receives the count used.
+ * Other arguments, outputs and errors as in qbsa_block_topk.
+ */
+qbsa_status qbsa_block_topk_keep(const float* q_mean, const float* k_mean, int B, int Nq, int Nkv, int nqb, int nkb,
+                                 int D, float scale, double keep, uint8_t* block_mask, float* block_scores,
+                                 int* n_keep_out, void* stream);
+
+/*
  * qbsa_wait_selftest -- test hook for failure detection (no counterpart on the source
  * pages): launches one thread that waits, through the same bounded mbarrier wait every
  * kernel of this library uses, on a phase that nothing ever completes.  After the wait
@@ -225,7 +247,8 @@ qbsa_status qbsa_check(void* stream);
 /* Thread-local description of the last non-OK status returned on this thread. */
 const char* qbsa_last_error(void);
 
-/* Library ABI version (major * 100 + minor): 101 (1.01 added qbsa_block_mean, qbsa_block_topk, qbsa_wait_selftest). */
+/* Library ABI version (major * 100 + minor): 102 (1.01 added qbsa_block_mean, qbsa_block_topk,
+ * qbsa_wait_selftest; 1.02 added qbsa_block_topk_keep). */
 int qbsa_version(void);
 
 #ifdef __cplusplus

@@ -15,7 +15,6 @@ from ._binding import (  # noqa: F401
     bsa_fwd,
     block_lists,
     estimate_block_mask,
-    keep_count,
     check,
     lib,
     qbsa_fwd,

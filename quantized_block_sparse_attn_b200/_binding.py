@@ -35,6 +35,7 @@ SIGNATURES = {
     "qbsa_block_lists": (_I, [_P, _I64, _I, _P, _P, _P]),
     "qbsa_block_mean": (_I, [_P, _I, _I, _I, _I, _P, _P]),
     "qbsa_block_topk": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P, _P, _P]),
+    "qbsa_block_topk_keep": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _F, ctypes.c_double, _P, _P, _P, _P]),
     "qbsa_wait_selftest": (_I, [_P]),
     "qbsa_check": (_I, [_P]),
     "qbsa_last_error": (ctypes.c_char_p, []),
@@ -369,25 +370,25 @@ def block_mean(x):
     return out
 
 
-def keep_count(n_kb: int, keep: float) -> int:
-    """Blocks kept per query block for a keep fraction: max(1, min(n_kb, round(keep * n_kb)))."""
-    return max(1, min(n_kb, int(round(keep * n_kb))))
-
-
 def block_topk(q_mean, k_mean, scale: float, *, keep: float = None, n_keep: int = None, return_scores: bool = False):
-    """Block mask (uint8 [B, Nq, nqb, nkb], 1 = compute) keeping the n_keep best pooled scores per query block."""
+    """Block mask (uint8 [B, Nq, nqb, nkb], 1 = compute) keeping the n_keep best pooled scores per query
+    block; with ``keep`` the library derives n_keep from the fraction (qbsa_block_topk_keep)."""
     import torch
     B, Nq, nqb, D = q_mean.shape
     Nkv, nkb = k_mean.shape[1], k_mean.shape[2]
-    if n_keep is None:
-        n_keep = keep_count(nkb, keep)
+    if (keep is None) == (n_keep is None):
+        raise ValueError("give exactly one of keep and n_keep")
     for t in (q_mean, k_mean):
         if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous():
             raise ValueError("q_mean and k_mean must be contiguous float32 CUDA tensors")
     mask = torch.empty((B, Nq, nqb, nkb), dtype=torch.uint8, device=q_mean.device)
     scores = torch.empty((B, Nq, nqb, nkb), dtype=torch.float32, device=q_mean.device) if return_scores else None
-    _ck(lib().qbsa_block_topk(_ptr(q_mean), _ptr(k_mean), B, Nq, Nkv, nqb, nkb, D, scale, n_keep, _ptr(mask),
-                              _ptr(scores), _stream(q_mean.device)))
+    if keep is not None:
+        _ck(lib().qbsa_block_topk_keep(_ptr(q_mean), _ptr(k_mean), B, Nq, Nkv, nqb, nkb, D, scale, float(keep),
+                                       _ptr(mask), _ptr(scores), None, _stream(q_mean.device)))
+    else:
+        _ck(lib().qbsa_block_topk(_ptr(q_mean), _ptr(k_mean), B, Nq, Nkv, nqb, nkb, D, scale, n_keep, _ptr(mask),
+                                  _ptr(scores), _stream(q_mean.device)))
     return (mask, scores) if return_scores else mask
 
 

@@ -124,7 +124,7 @@ qbsa_status launch_dense(qbsa::DenseParams& prm, int64_t n_work, cudaStream_t st
 
 extern "C" {
 
-int qbsa_version(void) { return 101; }
+int qbsa_version(void) { return 102; }
 
 const char* qbsa_last_error(void) { return g_last_error.c_str(); }
 
@@ -529,6 +529,17 @@ qbsa_status qbsa_block_topk(const float* q_mean, const float* k_mean, int B, int
                             static_cast<cudaStream_t>(stream)>>>(q_mean, k_mean, Nq, Nq / Nkv, nqb, nkb, D, scale,
                                                                   n_keep, block_mask, block_scores);
   return check_launch("block_topk_kernel launch");
+}
+
+qbsa_status qbsa_block_topk_keep(const float* q_mean, const float* k_mean, int B, int Nq, int Nkv, int nqb, int nkb,
+                                 int D, float scale, double keep, uint8_t* block_mask, float* block_scores,
+                                 int* n_keep_out, void* stream) {
+  if (!(keep >= 0.0 && keep <= 1.0)) return fail(QBSA_ERR_INVALID, "keep must be in [0, 1]");
+  if (nkb < 1) return fail(QBSA_ERR_INVALID, "sizes must be >= 1");
+  // blocks kept per query block: keep * nkb rounded to nearest (ties to even), at least 1
+  const int n_keep = std::max(1, std::min(nkb, static_cast<int>(std::nearbyint(keep * nkb))));
+  if (n_keep_out) *n_keep_out = n_keep;
+  return qbsa_block_topk(q_mean, k_mean, B, Nq, Nkv, nqb, nkb, D, scale, n_keep, block_mask, block_scores, stream);
 }
 
 namespace qbsa {

@@ -37,8 +37,6 @@ def heads_to_sequence(x: torch.Tensor, group=None) -> torch.Tensor:
     """[B, S/P, N, D] sequence slice -> [B, S, N/P, D]: rank r receives heads
     [r N/P, (r + 1) N/P) of every rank's slice, laid out in rank (= sequence) order."""
     world = dist.get_world_size(group)
-    if world == 1:
-        return x
     B, S_loc, N, D = x.shape
     if N % world != 0:
         raise ValueError(f"{N} heads are not divisible by {world} ranks")
@@ -53,8 +51,6 @@ def sequence_to_heads(y: torch.Tensor, group=None) -> torch.Tensor:
     """Inverse of heads_to_sequence: [B, S, N/P, D] -> [B, S/P, N, D] (rank r keeps sequence
     slice r of every rank's heads, laid out in rank (= head) order)."""
     world = dist.get_world_size(group)
-    if world == 1:
-        return y
     B, S, n, D = y.shape
     if S % world != 0:
         raise ValueError(f"sequence {S} is not divisible by {world} ranks")

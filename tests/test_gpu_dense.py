@@ -179,3 +179,48 @@ def test_bsa_parity(B, Nq, Nkv, S, D, keep):
                                               atten_mask=(el == 0).astype(np.uint8))
     compare_out(host_f64(out), ref, DENSE_MAX_ABS, DENSE_MEAN_ABS)
     compare_stats(smax.cpu().numpy(), ssum.cpu().numpy(), rmax, rsum)
+
+
+def _growing_k(k, Skv, factor=3.0):
+    """K tile j (128 keys) multiplied by 1 + factor * j.  With iid N(0,1) data and scale
+    D^-0.5 a row's max then grows by a median of about 11 log2 units per tile, past the
+    kernels' lazy-rescale threshold of 8: on the first test case every row rescales O in
+    TMEM at two to five of its tiles (3.3 on average)."""
+    from workloads import bf16_bits_to_f32
+    kf = bf16_bits_to_f32(k).copy()
+    for j in range(-(-Skv // 128)):
+        kf[:, :, j * 128:(j + 1) * 128] *= 1.0 + factor * j
+    return bf16_bits_from_f32(kf)
+
+
+@pytest.mark.parametrize("B,Nq,Nkv,Sq,Skv,D,mode,layout", [
+    (1, 2, 2, 256, 680, 128, 0, "BNSD"),    # two-tile kernel, one pair per head, short last K tile
+    (1, 3, 1, 650, 680, 128, 0, "BSND"),    # two-tile kernel, odd tile count
+    (1, 2, 1, 300, 680, 64, 0, "BNSD"),     # one-tile kernel (D = 64)
+    (1, 2, 1, 300, 680, 128, 3, "BNSD"),    # one-tile kernel (causal, bottom-right)
+])
+def test_dense_lazy_rescale_growing_k(B, Nq, Nkv, Sq, Skv, D, mode, layout):
+    """The rescale of O in TMEM (taken only when the running max grows by more than 2^8)
+    against the oracle, with every row's max growing past that threshold several times."""
+    q, k, v = _bnsd(13, B, Nq, Nkv, Sq, Skv, D)
+    k = _growing_k(k, Skv)
+    if layout == "BSND":
+        q, k, v = (np.ascontiguousarray(np.swapaxes(t, 1, 2)) for t in (q, k, v))
+    _run_and_compare(q, k, v, layout, Nq, D ** -0.5, mode)
+
+
+def test_bsa_lazy_rescale_growing_k():
+    """bsa_fwd (one-tile kernel walking a kept-block list) with the row max growing past the
+    rescale threshold at several kept K tiles."""
+    from workloads import block_keep_mask
+    B, Nq, Nkv, S, D = 1, 2, 1, 640, 128
+    q, k, v = _bnsd(14, B, Nq, Nkv, S, S, D)
+    k = _growing_k(k, S)
+    bm = block_keep_mask(14, B, Nq, 5, 5, 0.6)
+    out, smax, ssum = qb.bsa_fwd(dev_bf16(q), dev_bf16(k), dev_bf16(v), dev(bm), D ** -0.5)
+    qb.check()
+    el = np.repeat(np.repeat(bm, 128, axis=2), 128, axis=3)
+    ref, rmax, rsum = dense.attention_forward(q, k, v, layout="BNSD", scale=D ** -0.5,
+                                              atten_mask=(el == 0).astype(np.uint8))
+    compare_out(host_f64(out), ref, DENSE_MAX_ABS, DENSE_MEAN_ABS)
+    compare_stats(smax.cpu().numpy(), ssum.cpu().numpy(), rmax, rsum)

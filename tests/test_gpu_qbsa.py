@@ -7,7 +7,8 @@ import torch
 import quantized_block_sparse_attn_b200 as qb
 from oracle import dense, quant
 from workloads import CONFIGS, block_keep_mask, blocky_qk_bf16, iid_normal_bf16, random_atten_mask, sample_rows
-from tests.gpu_util import QUANT_MAX_ABS, compare_out, compare_stats, dev, dev_bf16, host_f64
+from oracle.formats import bf16_to_f64
+from tests.gpu_util import QUANT_MAX_ABS, check_qbsa, compare_out, dev, dev_bf16, host_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -40,9 +41,7 @@ def test_qbsa_parity_small(B, Nq, Nkv, Sq, Skv, keep):
     bm = block_keep_mask(20, B, Nq, -(-Sq // 128), -(-Skv // 128), keep)
     scale = D ** -0.5
     got, gmax, gsum = _run(q8, qs, k8, ks, v8, vs, bm, scale)
-    ref, rmax, rsum = quant.qbsa_forward(q8, k8, qs, ks, v8, vs, bm, scale)
-    compare_out(got, ref, QUANT_MAX_ABS)
-    compare_stats(gmax, gsum, rmax, rsum)
+    check_qbsa(got, gmax, gsum, q8, k8, qs, ks, v8, vs, bm, scale, tag=f"{Sq}x{Skv} keep {keep}:")
 
 
 @pytest.mark.parametrize("sign", [1.0, -1.0])
@@ -66,9 +65,7 @@ def test_qbsa_unequal_tile_pairs(sign):
     bm[0, 1, 1, :] = 1
     scale = sign * D ** -0.5
     got, gmax, gsum = _run(q8, qs, k8, ks, v8, vs, bm, scale)
-    ref, rmax, rsum = quant.qbsa_forward(q8, k8, qs, ks, v8, vs, bm, scale)
-    compare_out(got, ref, QUANT_MAX_ABS)
-    compare_stats(gmax, gsum, rmax, rsum)
+    check_qbsa(got, gmax, gsum, q8, k8, qs, ks, v8, vs, bm, scale, tag=f"unequal pairs sign {sign}:")
 
 
 @pytest.mark.parametrize("sign", [1.0, -1.0])
@@ -86,9 +83,7 @@ def test_qbsa_more_units_than_sms(sign):
     bm[1, 7, 2, :] = 0
     scale = sign * D ** -0.5
     got, gmax, gsum = _run(q8, qs, k8, ks, v8, vs, bm, scale)
-    ref, rmax, rsum = quant.qbsa_forward(q8, k8, qs, ks, v8, vs, bm, scale)
-    compare_out(got, ref, QUANT_MAX_ABS)
-    compare_stats(gmax, gsum, rmax, rsum, e4m3_flips=True)
+    check_qbsa(got, gmax, gsum, q8, k8, qs, ks, v8, vs, bm, scale, e4m3_flips=True, tag=f"waves sign {sign}:")
 
 
 @pytest.mark.parametrize("chunks", [1, 3, 8])
@@ -122,8 +117,7 @@ def test_qbsa_short_loops_repeated():
             q8, qs, k8, ks, v8, vs = _quantized(q, k, v)
             bm = np.ones((1, 1, S // 128, S // 128), dtype=np.uint8)
             got, gmax, gsum = _run(q8, qs, k8, ks, v8, vs, bm, D ** -0.5)
-            ref, rmax, rsum = quant.qbsa_forward(q8, k8, qs, ks, v8, vs, bm, D ** -0.5)
-            compare_out(got, ref, QUANT_MAX_ABS)
+            check_qbsa(got, gmax, gsum, q8, k8, qs, ks, v8, vs, bm, D ** -0.5, tag=f"S={S} rep {rep}:")
 
 
 def test_qbsa_empty_rows_and_zero_query_counts():
@@ -182,6 +176,8 @@ def test_quantisers_bit_exact(S):
 
 
 def _qbsa_workload(S, keep, heads_for_oracle, n_qblocks):
+    """One point of the Fig 4.1 workload (B=1, N=40, D=128), quantised on the GPU; sampled
+    heads and query blocks (first and last included) against both oracle readings."""
     c = CONFIGS["qbsa"]
     N, D, seed = c["Nq"], c["D"], c["seed"]
     q = blocky_qk_bf16(seed, "q", 1, N, S, D)
@@ -197,39 +193,52 @@ def _qbsa_workload(S, keep, heads_for_oracle, n_qblocks):
     qb.check()
     got, gmax, gsum = host_f64(out), smax.cpu().numpy(), ssum.cpu().numpy()
     qbs = sample_rows(seed, S, n_qblocks)
+    assert 0 in qbs and nb - 1 in qbs
     for h in heads_for_oracle:
         sl = (slice(0, 1), slice(h, h + 1))
         q8, qs, k8, ks, v8, vs = _quantized(q[sl], k[sl], v[sl])
         assert np.array_equal(tq8[0, h].cpu().numpy(), q8[0, 0])
         assert np.array_equal(tk8[0, h].cpu().numpy(), k8[0, 0])
         assert np.array_equal(tv8[0, h].cpu().numpy(), v8[0, 0])
+        assert np.array_equal(tqs[0, h].cpu().numpy().view(np.uint32), qs[0, 0].view(np.uint32))
+        assert np.array_equal(tks[0, h].cpu().numpy().view(np.uint32), ks[0, 0].view(np.uint32))
         assert np.array_equal(tvs[0, h].cpu().numpy().view(np.uint32), vs[0, 0].view(np.uint32))
-        ref, rmax, rsum = quant.qbsa_forward(q8, k8, qs, ks, v8, vs, bm[:, h:h + 1], c["scale"], q_blocks=qbs)
-        compare_out(got[:, h:h + 1], ref, QUANT_MAX_ABS)
-        compare_stats(gmax[:, h:h + 1], gsum[:, h:h + 1], rmax, rsum)
-        # reported, not gated: error against the unquantised attention over the same kept blocks
-        # (its element mask is S x S bytes, so only up to S = 64K)
-        if S > 65536:
-            continue
+        check_qbsa(got[:, h:h + 1], gmax[:, h:h + 1], gsum[:, h:h + 1], q8, k8, qs, ks, v8, vs, bm[:, h:h + 1],
+                   c["scale"], q_blocks=qbs, plain_max_abs=QUANT_MAX_ABS, tag=f"S={S} keep={keep} head {h}:")
+        # reported, not gated: error against the unquantised bf16 attention over the same kept blocks
         rows = np.concatenate([np.arange(b_ * 128, b_ * 128 + 128) for b_ in qbs])
-        keep_el = np.repeat(np.repeat(bm[0, h], 128, axis=0), 128, axis=1)
-        dref, _, _ = dense.attention_forward(q[sl], k[sl], v[sl], layout="BNSD", scale=c["scale"],
-                                             atten_mask=(keep_el == 0).astype(np.uint8), q_rows=rows)
-        e = np.abs(got[0, h, rows] - dref[0, 0, rows])
+        ok = np.repeat(bm[0, h][qbs], 128, axis=0)
+        ok = np.repeat(ok, 128, axis=1).astype(bool)
+        dref, _, _ = dense.attend(bf16_to_f64(q[0, h, rows]), bf16_to_f64(k[0, h]), bf16_to_f64(v[0, h]),
+                                  c["scale"], ok)
+        e = np.abs(got[0, h, rows] - dref)
         print(f"S={S} keep={keep} head {h}: error vs unquantised attention max {e.max():.3e} mean {e.mean():.3e}")
 
 
+# The ten points of the Fig 4.1 range (S from 8K to 128K, sparsity 0.9 and 0.5)
 @pytest.mark.parametrize("keep", [0.1, 0.5])
 def test_qbsa_workload_8k_sampled(keep):
     _qbsa_workload(8192, keep, heads_for_oracle=[0, 39], n_qblocks=6)
 
 
-@pytest.mark.slow
-def test_qbsa_workload_64k_sampled():
-    _qbsa_workload(65536, 0.1, heads_for_oracle=[0, 21], n_qblocks=4)
+@pytest.mark.parametrize("keep", [0.1, 0.5])
+def test_qbsa_workload_16k_sampled(keep):
+    _qbsa_workload(16384, keep, heads_for_oracle=[0, 17], n_qblocks=4)
+
+
+@pytest.mark.parametrize("keep", [0.1, 0.5])
+def test_qbsa_workload_32k_sampled(keep):
+    _qbsa_workload(32768, keep, heads_for_oracle=[5, 39], n_qblocks=3)
 
 
 @pytest.mark.slow
-def test_qbsa_workload_128k_keep_half_sampled():
-    """The largest configuration of the workload: S = 128K, half the blocks kept."""
-    _qbsa_workload(131072, 0.5, heads_for_oracle=[7], n_qblocks=2)
+@pytest.mark.parametrize("keep", [0.1, 0.5])
+def test_qbsa_workload_64k_sampled(keep):
+    _qbsa_workload(65536, keep, heads_for_oracle=[0, 21], n_qblocks=3)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("keep", [0.1, 0.5])
+def test_qbsa_workload_128k_sampled(keep):
+    """The largest configuration of the workload: S = 128K."""
+    _qbsa_workload(131072, keep, heads_for_oracle=[7], n_qblocks=2)

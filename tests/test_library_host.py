@@ -33,7 +33,27 @@ def test_every_declared_symbol_is_exported():
     raw = ctypes.CDLL(qb.LIB_PATH)
     for n in names:
         assert hasattr(raw, n), n
-    assert qb.lib().qbsa_version() == 101  # 1.01: block-mask estimation and the wait self-test added
+    assert qb.lib().qbsa_version() == 102  # 1.02: qbsa_block_topk_keep added
+
+
+@pytest.mark.parametrize("nkb", [1, 2, 5, 7, 64, 255, 512, 1024, 2048])
+@pytest.mark.parametrize("keep", [0.0, 0.05, 0.1, 0.25, 0.3, 0.5, 0.9, 1.0])
+def test_block_topk_keep_count_rule(nkb, keep):
+    """The kept-block count qbsa_block_topk_keep derives from a keep fraction equals the
+    oracle's rule; a null q_mean then stops the call before any launch."""
+    from oracle import estimate
+    n = ctypes.c_int(-1)
+    st = qb.lib().qbsa_block_topk_keep(None, None, 1, 1, 1, 1, nkb, 128, 0.1, keep, None, None, ctypes.byref(n),
+                                       None)
+    assert st == 1
+    assert n.value == estimate.keep_count(nkb, keep)
+
+
+@pytest.mark.parametrize("keep", [-0.1, 1.5, float("nan")])
+def test_block_topk_keep_rejects_bad_fraction(keep):
+    n = ctypes.c_int(-1)
+    st = qb.lib().qbsa_block_topk_keep(None, None, 1, 1, 1, 1, 8, 128, 0.1, keep, None, None, ctypes.byref(n), None)
+    assert st == 1 and n.value == -1
 
 
 def _attn(**over):
