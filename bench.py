@@ -4,9 +4,12 @@
 Default workload (one step = one qbsa_fwd call): quantized block-sparse attention,
 B=1, N=40, S=65536, D=128, INT8 Q/K per 128-token block, E4M3 V per channel, 128x128
 block mask keeping 10% of the blocks per (head, query block) with the diagonal kept.
-The dense bf16 video workload (attn_fwd, B=1, N=40, S=61440, D=128) is timed beside
-it and reported under "extra".  ``--sweep`` adds the S sweep 8K..128K at keep 0.1 and
-0.5 (and dense) as extra lines.
+Reported beside it under "extra": bf16 block-sparse attention on the same mask, the
+on-GPU quantisers, block-mask estimation, dense bf16 attention at S=61440 (the video
+workload) and S=65536, the causal (B=2, N=16, S=4096) and GQA varlen TND workloads,
+and the sweep over S = 8K..128K at keep 0.1 and 0.5 plus dense at each S (the metric's
+"vs S" curve; ``--no-sweep`` skips it).  Lines whose inputs fit in L2 flush it (a
+256 MB write) before every timed step and time each step alone.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -68,7 +71,7 @@ def parse():
     p.add_argument("--seq", type=int, default=65536)
     p.add_argument("--keep", type=float, default=0.1)
     p.add_argument("--dense-seq", type=int, default=61440)
-    p.add_argument("--sweep", action="store_true")
+    p.add_argument("--no-sweep", action="store_true")
     p.add_argument("--no-dense", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu", action="store_true")
@@ -177,8 +180,12 @@ def qbsa_work(inp):
     return executed, dense_eq, bytes_
 
 
-def time_steps(fn, steps: int, warmup: int, stream, dist=None, sampler=None):
-    """Run fn warmup times, then time exactly `steps` calls with CUDA events on `stream`."""
+def time_steps(fn, steps: int, warmup: int, stream, dist=None, sampler=None, flush=None):
+    """Run fn warmup times, then time exactly `steps` calls with CUDA events on `stream`.
+
+    With ``flush`` (a device buffer larger than L2) the buffer is overwritten before every
+    step, outside the events, so each step starts with a cold L2; the total is then the sum
+    of the per-step times."""
     import torch
     for _ in range(warmup):
         fn()
@@ -188,19 +195,37 @@ def time_steps(fn, steps: int, warmup: int, stream, dist=None, sampler=None):
     torch.cuda.synchronize()
     if sampler:
         sampler.start()
-    evs = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
-    evs[0].record(stream)
-    for i in range(steps):
-        fn()
-        evs[i + 1].record(stream)
+    if flush is None:
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+        evs[0].record(stream)
+        for i in range(steps):
+            fn()
+            evs[i + 1].record(stream)
+    else:
+        pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        for a, b in pairs:
+            flush.zero_()
+            a.record(stream)
+            fn()
+            b.record(stream)
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
     clocks = sampler.stop() if sampler else None
-    per = [evs[i].elapsed_time(evs[i + 1]) for i in range(steps)]
-    total = evs[0].elapsed_time(evs[-1])
+    if flush is None:
+        per = [evs[i].elapsed_time(evs[i + 1]) for i in range(steps)]
+        total = evs[0].elapsed_time(evs[-1])
+    else:
+        per = [a.elapsed_time(b) for a, b in pairs]
+        total = sum(per)
     return total, per, clocks
+
+
+def l2_flush_buffer(device):
+    """A 256 MB device buffer (twice the 126 MB L2) to overwrite between timed steps."""
+    import torch
+    return torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=device)
 
 
 def max_over_ranks(x: float, dist, device="cuda"):
@@ -371,7 +396,7 @@ def run_ours(args):
         h2d = sum(t.numel() * t.element_size() for t in host.values())
         host_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
         d2h = host_out.numel() * host_out.element_size()
-        e2e_steps = max(2, min(5, args.steps))
+        e2e_steps = max(2, min(10, args.steps))
 
         def e2e_step():
             res = qb.qbsa_fwd(host["q8"], host["k8"], host["qs"], host["ks"], host["v8"], host["vs"], host["bm"],
@@ -398,22 +423,33 @@ def run_ours(args):
                                 "sample": desc + f", {secs:.1f} s"}
 
     extra = {}
+    flush = l2_flush_buffer(device)
     # ---------------------------------------------------------------- bf16 block-sparse, same mask
     if not args.no_dense:
         extra["bsa_bf16_same_mask"] = bsa_line(device, stream, inp, executed, bf16_peak, ms_step)
     del inp
     torch.cuda.empty_cache()
+    # ---------------------------------------------------------------- on-GPU quantisers
+    extra["quantize"] = quantize_line(device, stream, args.seq, hbm_peak)
     # ---------------------------------------------------------------- block-mask estimation
     if not args.no_dense:
         extra["mask_estimation"] = estimate_line(device, stream, args.seq, args.keep, hbm_peak)
-    # ---------------------------------------------------------------- dense bf16 video workload
+    # ---------------------------------------------------------------- dense bf16
     if not args.no_dense:
-        extra["dense_video"] = dense_line(device, stream, args.dense_seq, max(2, args.warmup), 3, bf16_peak, dist)
-    if args.sweep:
+        extra["dense_video"] = dense_line(device, stream, args.dense_seq, max(2, args.warmup), 10, bf16_peak, dist)
+        extra["dense_S65536"] = dense_line(device, stream, 65536, 2, 10, bf16_peak, dist)
+        extra["causal"] = causal_line(device, stream, bf16_peak, flush)
+        extra["gqa_varlen"] = gqa_varlen_line(device, stream, bf16_peak, flush)
+    # ---------------------------------------------------------------- the metric's curve over S
+    if not args.no_sweep:
+        sweep = []
         for S in (8192, 16384, 32768, 65536, 131072):
             for keep in (0.1, 0.5):
-                extra[f"qbsa_S{S}_keep{keep}"] = qbsa_line(device, stream, S, keep, fp8_peak)
-            extra[f"dense_S{S}"] = dense_line(device, stream, S, 2, 3, bf16_peak, None)
+                sweep.append(qbsa_line(device, stream, S, keep, fp8_peak, flush if S <= 8192 else None))
+            if not args.no_dense:
+                sweep.append(dense_line(device, stream, S, 2, 3 if S > 65536 else 5, bf16_peak, None,
+                                        flush if S <= 8192 else None))
+        extra["sweep"] = sweep
     if extra:
         line["extra"] = extra
     if dist is not None:
@@ -424,7 +460,7 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
-def qbsa_line(device, stream, S, keep, fp8_peak):
+def qbsa_line(device, stream, S, keep, fp8_peak, flush=None):
     import torch
     import quantized_block_sparse_attn_b200 as qb
     inp = qbsa_inputs(S, keep, device)
@@ -435,12 +471,14 @@ def qbsa_line(device, stream, S, keep, fp8_peak):
         qb.qbsa_fwd(inp["q8"], inp["k8"], inp["qs"], inp["ks"], inp["v8"], inp["vs"], inp["bm"], inp["scale"],
                     out=out, return_stats=False)
 
-    total, per, _ = time_steps(step, 5, 2, stream)
-    ms = total / 5
+    total, per, _ = time_steps(step, 10, 2, stream, flush=flush)
+    qb.check(device)
+    ms = total / 10
     del inp
     torch.cuda.empty_cache()
-    return {"S": S, "keep": keep, "ms": ms, "executed_tflops": executed / ms / 1e9,
-            "dense_equivalent_tflops": dense_eq / ms / 1e9, "pct_of_fp8_peak": 100 * executed / ms / 1e9 / fp8_peak}
+    return {"kernel": "attn_qbsa_kernel", "S": S, "keep": keep, "ms": ms, "executed_tflops": executed / ms / 1e9,
+            "dense_equivalent_tflops": dense_eq / ms / 1e9, "pct_of_fp8_peak": 100 * executed / ms / 1e9 / fp8_peak,
+            "l2": "flushed before each step" if flush is not None else "inputs > L2"}
 
 
 def bsa_line(device, stream, inp, executed, bf16_peak, qbsa_ms):
@@ -457,9 +495,9 @@ def bsa_line(device, stream, inp, executed, bf16_peak, qbsa_ms):
     def step():
         qb.bsa_fwd(q, k, v, inp["bm"], inp["scale"], out=out, return_stats=False)
 
-    total, per, _ = time_steps(step, 5, 2, stream)
+    total, per, _ = time_steps(step, 10, 2, stream)
     qb.check(device)
-    ms = total / 5
+    ms = total / 10
     del q, k, v, out
     torch.cuda.empty_cache()
     return {"workload": f"bsa_fwd bf16 B=1 N=40 S={S} D=128, same block mask", "ms": ms,
@@ -503,7 +541,7 @@ def estimate_line(device, stream, S, keep, hbm_peak):
             "kernels": "block_mean_kernel x2 (HBM-bound), block_topk_kernel"}
 
 
-def dense_line(device, stream, S, warmup, steps, bf16_peak, dist):
+def dense_line(device, stream, S, warmup, steps, bf16_peak, dist, flush=None):
     import torch
     import quantized_block_sparse_attn_b200 as qb
     from workloads import CONFIGS, device_blocky_qk_bf16, device_iid_normal_bf16
@@ -517,14 +555,123 @@ def dense_line(device, stream, S, warmup, steps, bf16_peak, dist):
     def step():
         qb.attn_fwd(q, k, v, N, "BNSD", scale=c["scale"], out=out, return_stats=False)
 
-    total, per, clocks = time_steps(step, steps, warmup, stream, dist)
+    total, per, clocks = time_steps(step, steps, warmup, stream, dist, flush=flush)
     qb.check(device)
     ms = max_over_ranks(total / steps, dist)
     flops = 4.0 * D * S * S * N
     del q, k, v, out
     torch.cuda.empty_cache()
-    return {"workload": f"attn_fwd bf16 B=1 N=40 S={S} D=128 no mask", "ms": ms, "tflops": flops / ms / 1e9,
-            "pct_of_bf16_peak": 100 * flops / ms / 1e9 / bf16_peak, "kernel": "attn_pair_kernel"}
+    return {"workload": f"attn_fwd bf16 B=1 N=40 S={S} D=128 no mask", "S": S, "ms": ms, "tflops": flops / ms / 1e9,
+            "pct_of_bf16_peak": 100 * flops / ms / 1e9 / bf16_peak, "kernel": "attn_pair_kernel",
+            "l2": "flushed before each step" if flush is not None else "inputs > L2"}
+
+
+def _visited_tiles(sq: int, skv: int, mode: int) -> int:
+    """K tiles the kernel visits for one head of one sequence (the library's own schedule export)."""
+    import quantized_block_sparse_attn_b200 as qb
+    kb, ke, _, _ = qb.attn_tile_schedule(sq, skv, mode)
+    return int((ke - kb).sum())
+
+
+def causal_line(device, stream, bf16_peak, flush):
+    """The causal training-style workload: B=2, N=16, S=4096, D=128, BNSD, sparse_mode 3, with stats."""
+    import torch
+    import quantized_block_sparse_attn_b200 as qb
+    from workloads import CONFIGS, device_iid_normal_bf16
+    c = CONFIGS["causal"]
+    B, N, S, D, seed = c["B"], c["Nq"], c["S"], c["D"], c["seed"]
+    q, k, v = (device_iid_normal_bf16(seed, t, (B, N, S, D), device) for t in range(3))
+    out = torch.empty_like(q)
+    smax = torch.empty((B, N, S), dtype=torch.float32, device=device)
+    ssum = torch.empty_like(smax)
+
+    def step():
+        qb.attn_fwd(q, k, v, N, "BNSD", scale=c["scale"], sparse_mode=3, out=out, softmax_max=smax,
+                    softmax_sum=ssum)
+
+    total, per, _ = time_steps(step, 20, 3, stream, flush=flush)
+    qb.check(device)
+    ms = total / 20
+    executed = 4.0 * D * 128 * 128 * _visited_tiles(S, S, 3) * B * N
+    useful = 4.0 * D * (S * (S + 1) // 2) * B * N
+    del q, k, v, out, smax, ssum
+    torch.cuda.empty_cache()
+    return {"workload": f"attn_fwd bf16 causal (sparse_mode 3) B={B} N={N} S={S} D={D} BNSD, stats", "ms": ms,
+            "executed_tflops": executed / ms / 1e9, "useful_tflops": useful / ms / 1e9,
+            "pct_of_bf16_peak": 100 * executed / ms / 1e9 / bf16_peak, "kernel": "attn_dense_kernel<128>",
+            "l2": "flushed before each step"}
+
+
+def gqa_varlen_line(device, stream, bf16_peak, flush):
+    """The GQA varlen workload: TND, Nq=32, Nkv=8, D=128, sequences 1024/5000/10360, causal."""
+    import numpy as np
+    import torch
+    import quantized_block_sparse_attn_b200 as qb
+    from workloads import CONFIGS, device_iid_normal_bf16
+    c = CONFIGS["gqa_varlen"]
+    Nq, Nkv, D, seed, lens = c["Nq"], c["Nkv"], c["D"], c["seed"], c["seqlens"]
+    T = sum(lens)
+    cum = np.cumsum(lens).tolist()
+    q = device_iid_normal_bf16(seed, 0, (T, Nq, D), device)
+    k = device_iid_normal_bf16(seed, 1, (T, Nkv, D), device)
+    v = device_iid_normal_bf16(seed, 2, (T, Nkv, D), device)
+    out = torch.empty_like(q)
+
+    def step():
+        qb.attn_fwd(q, k, v, Nq, "TND", scale=c["scale"], sparse_mode=c["sparse_mode"], actual_seq_qlen=cum,
+                    actual_seq_kvlen=cum, out=out, return_stats=False)
+
+    total, per, _ = time_steps(step, 20, 3, stream, flush=flush)
+    qb.check(device)
+    ms = total / 20
+    executed = 4.0 * D * 128 * 128 * sum(_visited_tiles(n, n, 3) for n in lens) * Nq
+    useful = 4.0 * D * sum(n * (n + 1) // 2 for n in lens) * Nq
+    del q, k, v, out
+    torch.cuda.empty_cache()
+    return {"workload": f"attn_fwd bf16 TND GQA Nq={Nq} Nkv={Nkv} D={D} lengths {list(lens)} causal", "ms": ms,
+            "executed_tflops": executed / ms / 1e9, "useful_tflops": useful / ms / 1e9,
+            "pct_of_bf16_peak": 100 * executed / ms / 1e9 / bf16_peak, "kernel": "attn_dense_kernel<128>",
+            "l2": "flushed before each step"}
+
+
+def quantize_line(device, stream, S, hbm_peak):
+    """The on-GPU quantisers on the quantized workload's bf16 Q/K/V at this S (HBM-bound)."""
+    import torch
+    import quantized_block_sparse_attn_b200 as qb
+    from workloads import CONFIGS, device_blocky_qk_bf16, device_iid_normal_bf16
+    c = CONFIGS["qbsa"]
+    N, D, seed = c["Nq"], c["D"], c["seed"]
+    q = device_blocky_qk_bf16(seed, "q", 1, N, S, D, device)
+    v = device_iid_normal_bf16(seed, 2, (1, N, S, D), device)
+    nb = -(-S // 128)
+    codes = torch.empty((1, N, S, D), dtype=torch.int8, device=device)
+    qsc = torch.empty((1, N, nb), dtype=torch.float32, device=device)
+    vcodes = torch.empty((1, N, S, D), dtype=torch.uint8, device=device)
+    vsc = torch.empty((1, N, D), dtype=torch.float32, device=device)
+    L = qb.lib()
+    from quantized_block_sparse_attn_b200._binding import _ptr, _stream
+
+    def qk():
+        L.qbsa_quantize_qk(_ptr(q), 1, N, S, D, _ptr(codes), _ptr(qsc), _stream(device))
+
+    def vq():
+        L.qbsa_quantize_v(_ptr(v), 1, N, S, D, _ptr(vcodes), _ptr(vsc), _stream(device))
+
+    qk_ms, _, _ = time_steps(qk, 10, 3, stream)
+    v_ms, _, _ = time_steps(vq, 10, 3, stream)
+    qb.check(device)
+    qk_ms, v_ms = qk_ms / 10, v_ms / 10
+    qk_bytes = N * S * D * 2 + N * S * D + N * nb * 4
+    v_bytes = N * S * D * 2 + N * S * D + N * D * 4
+    del q, v, codes, vcodes
+    torch.cuda.empty_cache()
+    return {"workload": f"quantisers B=1 N=40 S={S} D=128 (one tensor each)",
+            "qk_ms": qk_ms, "qk_gbs": qk_bytes / (qk_ms / 1e3) / 1e9,
+            "qk_frac_of_hbm": qk_bytes / (qk_ms / 1e3) / 1e9 / hbm_peak,
+            "v_ms": v_ms, "v_gbs": v_bytes / (v_ms / 1e3) / 1e9,
+            "v_frac_of_hbm": v_bytes / (v_ms / 1e3) / 1e9 / hbm_peak,
+            "algorithmic_bytes": "bf16 read once + 8-bit codes and fp32 scales written once",
+            "kernels": "quantize_qk_kernel<128>, v_quant_kernel<128> (one pass over HBM, re-read from L2)"}
 
 
 def main():

@@ -12,7 +12,9 @@
  * Conventions for every entry point:
  *   - The caller owns all memory.  Device pointers must be 16-byte aligned and stay
  *     valid until the work queued on `stream` has finished; the library never frees
- *     or retains them and allocates no device memory of its own.
+ *     or retains them.  Only qbsa_quantize_v takes scratch memory of its own, from
+ *     the stream-ordered allocator on `stream` (see there); no other entry point
+ *     allocates device memory.
  *   - Work is queued asynchronously on `stream` (a cudaStream_t; NULL = legacy default
  *     stream).  Argument checks run on the host before anything is queued: a
  *     non-OK status means nothing was launched.
@@ -152,6 +154,7 @@ qbsa_status qbsa_fwd(const int8_t* q_i8, const int8_t* k_i8, const float* q_bloc
  * ([QBSA] "EagleQBSA量化叠加稀疏方案设计"): for each (b, h, block) a = max|x| (fp32),
  * s = a/127 (1 if a = 0), codes = rint_half_even(x/s) clamped to [-127, 127].
  * x bf16 [B, N, S, D] (BNSD); codes int8 [B, N, S, D]; scales fp32 [B, N, ceil(S/128)].
+ * D in {64, 128, 256} (else QBSA_ERR_UNSUPPORTED); x and codes 16-byte aligned.
  */
 qbsa_status qbsa_quantize_qk(const void* x_bf16, int B, int N, int S, int D, int8_t* codes, float* scales,
                              void* stream);
@@ -160,7 +163,14 @@ qbsa_status qbsa_quantize_qk(const void* x_bf16, int B, int N, int S, int D, int
  * qbsa_quantize_v -- per-channel FP8 E4M3 quantisation of V ([QBSA] same section):
  * for each (b, h, channel c) a = max over the sequence of |v[:, c]|, s_c = a/448 (1 if
  * a = 0), codes = e4m3_rne_satfinite(v / s_c).  v bf16 [B, N, S, D]; codes [B, N, S, D];
- * scales fp32 [B, N, D] (also used as the running max while the call is in flight).
+ * scales fp32 [B, N, D].  D in {64, 128, 256} (else QBSA_ERR_UNSUPPORTED); v, codes and
+ * scales 16-byte aligned.
+ * One kernel pass reads V once from HBM: each head's column maxima are gathered first and
+ * its codes written right after, while the head is still in L2.  The pass needs
+ * (1 + B*N*(D+1)) * 4 bytes of scratch (work-item counter, per-head arrival counters and
+ * column maxima), which this call takes from the stream-ordered allocator
+ * (cudaMallocAsync / cudaFreeAsync on `stream`, the device's current memory pool) and
+ * zeroes; an allocation failure returns QBSA_ERR_CUDA before the kernel is queued.
  */
 qbsa_status qbsa_quantize_v(const void* v_bf16, int B, int N, int S, int D, uint8_t* codes, float* scales,
                             void* stream);

@@ -424,34 +424,100 @@ qbsa_status qbsa_quantize_qk(const void* x_bf16, int B, int N, int S, int D, int
                              void* stream) {
   if (!x_bf16 || !codes || !scales) return fail(QBSA_ERR_INVALID, "null pointer");
   if (B < 1 || N < 1 || S < 1 || D < 1) return fail(QBSA_ERR_INVALID, "B, N, S, D must be >= 1");
+  if (D != 64 && D != 128 && D != 256) return fail(QBSA_ERR_UNSUPPORTED, "D must be 64, 128 or 256 (got %d)", D);
+  if (!aligned16(x_bf16) || !aligned16(codes)) return fail(QBSA_ERR_INVALID, "x and codes must be 16-byte aligned");
+  if (S > kMaxLen) return fail(QBSA_ERR_UNSUPPORTED, "sequence length above %lld", (long long)kMaxLen);
   const int nblk = (S + 127) / 128;
-  if (nblk > 0x7fffffff || N > 65535 || B > 65535) return fail(QBSA_ERR_UNSUPPORTED, "grid too large");
-  qbsa::quantize_qk_kernel<<<dim3(nblk, N, B), 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      static_cast<const __nv_bfloat16*>(x_bf16), N, S, D, codes, scales);
+  if (N > 65535 || B > 65535) return fail(QBSA_ERR_UNSUPPORTED, "grid too large");
+  const dim3 grid(nblk, N, B);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(x_bf16);
+  if (D == 64) qbsa::quantize_qk_kernel<64><<<grid, qbsa::kQuantThreads, 0, st>>>(x, N, S, codes, scales);
+  else if (D == 128) qbsa::quantize_qk_kernel<128><<<grid, qbsa::kQuantThreads, 0, st>>>(x, N, S, codes, scales);
+  else qbsa::quantize_qk_kernel<256><<<grid, qbsa::kQuantThreads, 0, st>>>(x, N, S, codes, scales);
   return check_launch("quantize_qk_kernel launch");
 }
 
-qbsa_status qbsa_quantize_v(const void* v_bf16, int B, int N, int S, int D, uint8_t* codes, float* scales,
-                            void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Scratch of the V quantiser: ticket, per-head arrival counters, per-head column maxima.
+int64_t v_quant_scratch_words(int64_t H, int D) { return 1 + H + H * D; }
+
+// Validates the V quantiser's arguments; on success fills the launch parameters (scratch
+// pointers excluded) and the persistent grid size.
+qbsa_status v_quant_setup(const void* v_bf16, int B, int N, int S, int D, uint8_t* codes, float* scales,
+                          qbsa::VQuantParams* prm, unsigned* grid) {
   if (!v_bf16 || !codes || !scales) return fail(QBSA_ERR_INVALID, "null pointer");
   if (B < 1 || N < 1 || S < 1 || D < 1) return fail(QBSA_ERR_INVALID, "B, N, S, D must be >= 1");
-  if (D % 2 != 0 || D > 1024) return fail(QBSA_ERR_UNSUPPORTED, "D must be even and <= 1024");
-  if (N > 65535 || B > 65535) return fail(QBSA_ERR_UNSUPPORTED, "grid too large");
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int64_t nsc = (int64_t)B * N * D;
-  cudaError_t e = cudaMemsetAsync(scales, 0, nsc * sizeof(float), s);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
-  const int rows_per_cta = 256;
-  qbsa::v_colmax_kernel<<<dim3((S + rows_per_cta - 1) / rows_per_cta, N, B), D, 0, s>>>(
-      static_cast<const __nv_bfloat16*>(v_bf16), N, S, D, rows_per_cta, reinterpret_cast<unsigned int*>(scales));
-  qbsa_status st = check_launch("v_colmax_kernel launch");
-  if (st != QBSA_OK) return st;
-  qbsa::v_scale_kernel<<<(unsigned)((nsc + 255) / 256), 256, 0, s>>>(scales, (int)nsc);
-  if ((st = check_launch("v_scale_kernel launch")) != QBSA_OK) return st;
-  const int64_t total = (int64_t)B * N * S * D;
-  qbsa::v_quant_kernel<<<148 * 8, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(v_bf16), N, S, D, scales, codes,
-                                                total);
+  if (D != 64 && D != 128 && D != 256) return fail(QBSA_ERR_UNSUPPORTED, "D must be 64, 128 or 256 (got %d)", D);
+  if (!aligned16(v_bf16) || !aligned16(codes) || !aligned16(scales))
+    return fail(QBSA_ERR_INVALID, "v, codes and scales must be 16-byte aligned");
+  if (S > kMaxLen) return fail(QBSA_ERR_UNSUPPORTED, "sequence length above %lld", (long long)kMaxLen);
+  const int rows = D == 64 ? qbsa::VQuantCfg<64>::kRows : D == 128 ? qbsa::VQuantCfg<128>::kRows
+                                                                   : qbsa::VQuantCfg<256>::kRows;
+  const int64_t H = (int64_t)B * N;
+  const int64_t n_ch = (S + rows - 1) / rows;
+  if (2 * H * n_ch > 0xffffffffLL - 4 * 1024 * 1024 || H > 0x7fffffffLL)
+    return fail(QBSA_ERR_UNSUPPORTED, "too many (head, chunk) work items");
+  memset(prm, 0, sizeof(*prm));
+  prm->v = static_cast<const __nv_bfloat16*>(v_bf16);
+  prm->codes = codes;
+  prm->scales = scales;
+  prm->H = static_cast<int>(H);
+  prm->S = S;
+  prm->n_ch = static_cast<int>(n_ch);
+  prm->total = static_cast<unsigned int>(2 * H * n_ch);
+  int dev = 0, sms = 0, per_sm = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e == cudaSuccess) {
+    e = D == 64 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, qbsa::v_quant_kernel<64>, qbsa::kQuantThreads, 0)
+        : D == 128 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, qbsa::v_quant_kernel<128>, qbsa::kQuantThreads, 0)
+                   : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, qbsa::v_quant_kernel<256>, qbsa::kQuantThreads, 0);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "querying the SM count / occupancy");
+  *grid = static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>((int64_t)sms * std::max(per_sm, 1), prm->total)));
+  return QBSA_OK;
+}
+
+qbsa_status v_quant_launch(const qbsa::VQuantParams& prm, int D, unsigned grid, cudaStream_t st) {
+  if (D == 64) qbsa::v_quant_kernel<64><<<grid, qbsa::kQuantThreads, 0, st>>>(prm);
+  else if (D == 128) qbsa::v_quant_kernel<128><<<grid, qbsa::kQuantThreads, 0, st>>>(prm);
+  else qbsa::v_quant_kernel<256><<<grid, qbsa::kQuantThreads, 0, st>>>(prm);
   return check_launch("v_quant_kernel launch");
+}
+
+}  // namespace
+
+extern "C" {
+
+qbsa_status qbsa_quantize_v(const void* v_bf16, int B, int N, int S, int D, uint8_t* codes, float* scales,
+                            void* stream) {
+  qbsa::VQuantParams prm;
+  unsigned grid = 0;
+  qbsa_status st = v_quant_setup(v_bf16, B, N, S, D, codes, scales, &prm, &grid);
+  if (st != QBSA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t bytes = static_cast<size_t>(v_quant_scratch_words(prm.H, D)) * sizeof(unsigned int);
+  void* scratch = nullptr;
+  cudaError_t e = cudaMallocAsync(&scratch, bytes, s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMallocAsync (V quantiser scratch)");
+  e = cudaMemsetAsync(scratch, 0, bytes, s);
+  if (e != cudaSuccess) {
+    cudaFreeAsync(scratch, s);
+    return cuda_fail(e, "cudaMemsetAsync (V quantiser scratch)");
+  }
+  unsigned int* w = static_cast<unsigned int*>(scratch);
+  prm.ticket = w;
+  prm.arrived = w + 1;
+  prm.amax = w + 1 + prm.H;
+  st = v_quant_launch(prm, D, grid, s);
+  e = cudaFreeAsync(scratch, s);
+  if (st != QBSA_OK) return st;
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFreeAsync (V quantiser scratch)");
+  return QBSA_OK;
 }
 
 // ------------------------------------------------------------------------------

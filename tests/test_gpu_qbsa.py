@@ -158,21 +158,41 @@ def test_block_lists_hook_bit_exact():
             assert np.all(lists[r, len(idx):] == -1)
 
 
-@pytest.mark.parametrize("S", [300, 4096])
-def test_quantisers_bit_exact(S):
-    B, N, D = 2, 3, 128
+@pytest.mark.parametrize("B,N,S,D", [
+    (2, 3, 300, 128),       # ragged 128-row block; V: one chunk per head
+    (2, 3, 4096, 128),      # V: 16 chunks per head, pass 2 of a head interleaved with pass 1 of the next
+    (1, 1, 100, 128),       # a single head and a single short chunk
+    (1, 5, 1000, 64),
+    (3, 2, 777, 256),
+    (1, 2, 40000, 128),     # 157 chunks per head, ragged last chunk
+])
+def test_quantisers_bit_exact(B, N, S, D):
     x = blocky_qk_bf16(23, "q", B, N, S, D)
     v = iid_normal_bf16(23, 2, B, N, S, D)
-    v[0, 1, :, 5] = 0  # an all-zero channel takes scale 1
+    v[0, N - 1, :, 5] = 0  # an all-zero channel takes scale 1
     c8, cs = qb.quantize_qk(dev_bf16(x))
     v8, vs = qb.quantize_v(dev_bf16(v))
-    torch.cuda.synchronize()
+    qb.check()
     r8, rs = quant.quantize_qk_per_block(x)
     rv8, rvs = quant.quantize_v_per_channel(v)
     assert np.array_equal(c8.cpu().numpy(), r8)
     assert np.array_equal(cs.cpu().numpy().view(np.uint32), rs.view(np.uint32))
     assert np.array_equal(vs.cpu().numpy().view(np.uint32), rvs.view(np.uint32))
     assert np.array_equal(v8.cpu().numpy(), rv8)
+
+
+def test_quantise_v_repeated_calls():
+    """The V quantiser's scratch (ticket, arrival counters, column maxima) starts from zero on
+    every call: the same input twice, then a different one, give the oracle's bytes each time."""
+    B, N, S, D = 1, 4, 3000, 128
+    v1 = iid_normal_bf16(26, 2, B, N, S, D)
+    v2 = iid_normal_bf16(27, 2, B, N, S, D)
+    for v in (v1, v1, v2):
+        v8, vs = qb.quantize_v(dev_bf16(v))
+        qb.check()
+        rv8, rvs = quant.quantize_v_per_channel(v)
+        assert np.array_equal(v8.cpu().numpy(), rv8)
+        assert np.array_equal(vs.cpu().numpy().view(np.uint32), rvs.view(np.uint32))
 
 
 def _qbsa_workload(S, keep, heads_for_oracle, n_qblocks):

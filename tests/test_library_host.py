@@ -160,3 +160,20 @@ def test_tile_schedule_matches_oracle_sets(sq, skv, mode, pre, nxt):
         got_part = [x for x in got_vis if not (fb[t] <= x < fe[t])]
         assert got_vis == vis, (t, got_vis, vis)
         assert got_part == part, (t, got_part, part)
+
+
+@pytest.mark.parametrize("fn", ["qbsa_quantize_qk", "qbsa_quantize_v"])
+@pytest.mark.parametrize("over,status", [
+    (dict(x=None), 1),
+    (dict(x=ctypes.c_void_p(0x10002)), 1),
+    (dict(codes=ctypes.c_void_p(0x10008)), 1),
+    (dict(D=96), 2),
+    (dict(D=0), 1),
+    (dict(S=0), 1),
+])
+def test_quantisers_reject_before_launch(fn, over, status):
+    fake = ctypes.c_void_p(0x10000)
+    a = dict(x=fake, B=1, N=2, S=256, D=128, codes=fake, scales=fake)
+    a.update(over)
+    st = getattr(qb.lib(), fn)(a["x"], a["B"], a["N"], a["S"], a["D"], a["codes"], a["scales"], None)
+    assert st == status, qb.lib().qbsa_last_error().decode()
