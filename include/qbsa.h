@@ -176,6 +176,27 @@ qbsa_status qbsa_quantize_v(const void* v_bf16, int B, int N, int S, int D, uint
                             void* stream);
 
 /*
+ * qbsa_quantize_v_noalloc -- qbsa_quantize_v for callers that cannot allocate device
+ * memory during the call.  The source pages have no counterpart: this entry point exists
+ * for callers such as code running inside a custom allocator or a memory-pool callback,
+ * serving processes that reserve every byte of the device heap up front, and runtimes
+ * that forbid cudaMalloc / cudaMallocAsync on their streams.  It produces the same codes
+ * and scales as qbsa_quantize_v (same arguments, layouts and errors) and allocates
+ * nothing: its scratch (work-item counter, per-head arrival counters, per-head column
+ * maxima: 1 + B*N*(D+1) 32-bit words) lives in a fixed 256 KiB array in the library's
+ * device image, which every device that loads the library holds until the process exits.
+ *   - B*N*(D+1) + 1 above 65536 words (for D = 128: B*N above 507) returns
+ *     QBSA_ERR_UNSUPPORTED before anything is queued.
+ *   - The first call on a device looks up the array's device address for that device
+ *     (cudaGetSymbolAddress) and keeps it; make that first call before any stream capture.
+ *   - Every call zeroes the array with cudaMemsetAsync on `stream` and then reuses it, so
+ *     calls whose work overlaps on the GPU (other streams, other host threads) race on the
+ *     shared array: serialise them.
+ */
+qbsa_status qbsa_quantize_v_noalloc(const void* v_bf16, int B, int N, int S, int D, uint8_t* codes, float* scales,
+                                    void* stream);
+
+/*
  * attn_tile_schedule -- host-only export of the K-tile schedule attn_fwd's kernel uses
  * for one sequence under sparse_mode / pre_tokens / next_tokens ([NFA] §4.3): for each
  * 128-row query tile t < n_qtiles (= ceil(sq/128)), the K tiles [kt_begin[t],

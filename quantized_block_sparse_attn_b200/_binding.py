@@ -31,6 +31,7 @@ SIGNATURES = {
     "bsa_fwd": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P]),
     "qbsa_quantize_qk": (_I, [_P, _I, _I, _I, _I, _P, _P, _P]),
     "qbsa_quantize_v": (_I, [_P, _I, _I, _I, _I, _P, _P, _P]),
+    "qbsa_quantize_v_noalloc": (_I, [_P, _I, _I, _I, _I, _P, _P, _P]),
     "attn_tile_schedule": (_I, [_I64, _I64, _I, _I64, _I64, _P, _P, _P, _P, _I64]),
     "qbsa_block_lists": (_I, [_P, _I64, _I, _P, _P, _P]),
     "qbsa_block_mean": (_I, [_P, _I, _I, _I, _I, _P, _P]),

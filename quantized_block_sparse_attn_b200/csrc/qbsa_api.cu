@@ -5,6 +5,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <numeric>
 #include <string>
 #include <vector>
@@ -519,6 +520,76 @@ qbsa_status qbsa_quantize_v(const void* v_bf16, int B, int N, int S, int D, uint
   if (e != cudaSuccess) return cuda_fail(e, "cudaFreeAsync (V quantiser scratch)");
   return QBSA_OK;
 }
+
+}  // extern "C"
+
+// ------------------------------------------------------------------------------
+// V quantiser with a library-resident scratch array (no allocation per call)
+// ------------------------------------------------------------------------------
+//
+// Some callers cannot allocate device memory at the moment they quantise V: code that
+// runs inside a custom allocator or a memory-pool callback, callers whose device heap is
+// fully reserved up front (a serving process that pre-plans every byte), or runtimes
+// that forbid cudaMalloc / cudaMallocAsync on their streams.  This entry point gives them
+// the same V quantiser with its scratch (ticket counter, per-head arrival counters and
+// per-head column maxima) in a fixed array that lives in the library's device image.
+
+namespace {
+
+constexpr int64_t kNoAllocScratchWords = 65536;  // 256 KiB per device, held until the process exits
+__device__ __align__(256) unsigned int g_vq_scratch[kNoAllocScratchWords];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_vq_scratch_mu;
+unsigned int* g_vq_scratch_ptr[kMaxDevices] = {};
+
+// Device address of g_vq_scratch on the current device, looked up once per device (in
+// host code the symbol is only a host-side stand-in, never a device address).
+qbsa_status vq_scratch_address(unsigned int** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(QBSA_ERR_UNSUPPORTED, "device ordinal %d above %d", dev, kMaxDevices);
+  std::lock_guard<std::mutex> lock(g_vq_scratch_mu);
+  if (!g_vq_scratch_ptr[dev]) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_vq_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress (V quantiser scratch)");
+    g_vq_scratch_ptr[dev] = static_cast<unsigned int*>(ptr);
+  }
+  *out = g_vq_scratch_ptr[dev];
+  return QBSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+qbsa_status qbsa_quantize_v_noalloc(const void* v_bf16, int B, int N, int S, int D, uint8_t* codes, float* scales,
+                                    void* stream) {
+  qbsa::VQuantParams prm;
+  unsigned grid = 0;
+  qbsa_status st = v_quant_setup(v_bf16, B, N, S, D, codes, scales, &prm, &grid);
+  if (st != QBSA_OK) return st;
+  const int64_t words = v_quant_scratch_words(prm.H, D);
+  if (words > kNoAllocScratchWords)
+    return fail(QBSA_ERR_UNSUPPORTED,
+                "qbsa_quantize_v_noalloc: B*N*(D+1)+1 = %lld scratch words exceed the fixed %lld (256 KiB); "
+                "use qbsa_quantize_v", (long long)words, (long long)kNoAllocScratchWords);
+  unsigned int* w = nullptr;
+  if ((st = vq_scratch_address(&w)) != QBSA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(w, 0, static_cast<size_t>(words) * sizeof(unsigned int), s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync (V quantiser scratch)");
+  prm.ticket = w;
+  prm.arrived = w + 1;
+  prm.amax = w + 1 + prm.H;
+  return v_quant_launch(prm, D, grid, s);
+}
+
+}  // extern "C"
+
+extern "C" {
 
 // ------------------------------------------------------------------------------
 // schedule export, mask compaction hook, error word
