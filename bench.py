@@ -40,7 +40,7 @@ FP8_OVER_BF16 = 2.0  # nominal dense ratio (4.5 vs 2.25 PFLOP/s), applied to the
 # identified by their sha1.
 QBSA_NCU_TRAFFIC = {"sources": {"quantized_block_sparse_attn_b200/csrc/attn_qbsa.cuh": "5a21fd90ccb9d35f74b4398bc7764686c1cf59fe",
                                 "quantized_block_sparse_attn_b200/csrc/ptx_sm100.cuh": "76287e5abe014dfeeab1944e7be8a2564b0e0057"},
-                    "seq": 16384, "keep": 0.1, "bytes": 456649216, "alg_bytes": 420147200}
+                    "seq": 16384, "keep": 0.1, "bytes": 459491584, "alg_bytes": 420147200}
 
 
 def qbsa_traffic(seq: int, keep: float, alg_bytes: int):
@@ -598,7 +598,7 @@ def causal_line(device, stream, bf16_peak, flush):
     torch.cuda.empty_cache()
     return {"workload": f"attn_fwd bf16 causal (sparse_mode 3) B={B} N={N} S={S} D={D} BNSD, stats", "ms": ms,
             "executed_tflops": executed / ms / 1e9, "useful_tflops": useful / ms / 1e9,
-            "pct_of_bf16_peak": 100 * executed / ms / 1e9 / bf16_peak, "kernel": "attn_dense_kernel<128>",
+            "pct_of_bf16_peak": 100 * executed / ms / 1e9 / bf16_peak, "kernel": "attn_pair_masked_kernel",
             "l2": "flushed before each step"}
 
 
@@ -630,7 +630,7 @@ def gqa_varlen_line(device, stream, bf16_peak, flush):
     torch.cuda.empty_cache()
     return {"workload": f"attn_fwd bf16 TND GQA Nq={Nq} Nkv={Nkv} D={D} lengths {list(lens)} causal", "ms": ms,
             "executed_tflops": executed / ms / 1e9, "useful_tflops": useful / ms / 1e9,
-            "pct_of_bf16_peak": 100 * executed / ms / 1e9 / bf16_peak, "kernel": "attn_dense_kernel<128>",
+            "pct_of_bf16_peak": 100 * executed / ms / 1e9 / bf16_peak, "kernel": "attn_pair_masked_kernel",
             "l2": "flushed before each step"}
 
 

@@ -165,12 +165,12 @@ qbsa_status qbsa_quantize_qk(const void* x_bf16, int B, int N, int S, int D, int
  * a = 0), codes = e4m3_rne_satfinite(v / s_c).  v bf16 [B, N, S, D]; codes [B, N, S, D];
  * scales fp32 [B, N, D].  D in {64, 128, 256} (else QBSA_ERR_UNSUPPORTED); v, codes and
  * scales 16-byte aligned.
- * One kernel pass reads V once from HBM: each head's column maxima are gathered first and
- * its codes written right after, while the head is still in L2.  The pass needs
- * (1 + B*N*(D+1)) * 4 bytes of scratch (work-item counter, per-head arrival counters and
- * column maxima), which this call takes from the stream-ordered allocator
- * (cudaMallocAsync / cudaFreeAsync on `stream`, the device's current memory pool) and
- * zeroes; an allocation failure returns QBSA_ERR_CUDA before the kernel is queued.
+ * Two streaming passes: the column maxima of every (head, chunk), folded per head, then
+ * the codes (heads in reverse order, so the first chunks read are still in L2).  They need
+ * B*N*D * 4 bytes of scratch for the per-head maxima, which this call takes from the
+ * stream-ordered allocator (cudaMallocAsync / cudaFreeAsync on `stream`, the device's
+ * current memory pool) and zeroes; an allocation failure returns QBSA_ERR_CUDA before the
+ * kernels are queued.
  */
 qbsa_status qbsa_quantize_v(const void* v_bf16, int B, int N, int S, int D, uint8_t* codes, float* scales,
                             void* stream);
@@ -182,11 +182,11 @@ qbsa_status qbsa_quantize_v(const void* v_bf16, int B, int N, int S, int D, uint
  * serving processes that reserve every byte of the device heap up front, and runtimes
  * that forbid cudaMalloc / cudaMallocAsync on their streams.  It produces the same codes
  * and scales as qbsa_quantize_v (same arguments, layouts and errors) and allocates
- * nothing: its scratch (work-item counter, per-head arrival counters, per-head column
- * maxima: 1 + B*N*(D+1) 32-bit words) lives in a fixed 256 KiB array in the library's
- * device image, which every device that loads the library holds until the process exits.
- *   - B*N*(D+1) + 1 above 65536 words (for D = 128: B*N above 507) returns
- *     QBSA_ERR_UNSUPPORTED before anything is queued.
+ * nothing: its scratch (the per-head column maxima: B*N*D 32-bit words) lives in a fixed
+ * 256 KiB array in the library's device image, which every device that loads the library
+ * holds until the process exits.
+ *   - B*N*D above 65536 words (for D = 128: B*N above 512) returns QBSA_ERR_UNSUPPORTED
+ *     before anything is queued.
  *   - The first call on a device looks up the array's device address for that device
  *     (cudaGetSymbolAddress) and keeps it; make that first call before any stream capture.
  *   - Every call zeroes the array with cudaMemsetAsync on `stream` and then reuses it, so

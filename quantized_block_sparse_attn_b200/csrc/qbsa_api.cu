@@ -16,6 +16,7 @@
 #include "../../include/qbsa.h"
 #include "attn_dense.cuh"
 #include "attn_pair.cuh"
+#include "attn_pair_masked.cuh"
 #include "attn_qbsa.cuh"
 #include "estimate.cuh"
 #include "quantize.cuh"
@@ -321,6 +322,62 @@ static qbsa_status attn_fwd_impl(const void* q, const void* k, const void* v, in
                              s>>>(pp);
     return check_launch("attn_pair_kernel launch");
   }
+  // D = 128 under band / causal masks or TND, without an explicit atten_mask, pse or block
+  // mask: two query tiles per CTA with their own K-tile ranges
+  const bool pair_masked_path = D == 128 && !atten_mask && !pse && !block_mask;
+  if (pair_masked_path) {
+    qbsa::PairMaskedParams pp;
+    memset(&pp, 0, sizeof(pp));
+    pp.tm_q = prm.tm_q;
+    pp.tm_k = prm.tm_k;
+    pp.tm_v = prm.tm_v;
+    if (!tnd &&
+        (st = make_map(&pp.tm_o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, attention_out, qd, qs, 64)) != QBSA_OK)
+      return st;
+    pp.out = static_cast<__nv_bfloat16*>(attention_out);
+    pp.softmax_max = softmax_max;
+    pp.softmax_sum = softmax_sum;
+    pp.o_row_stride = prm.o_row_stride;
+    pp.o_head_stride = prm.o_head_stride;
+    pp.stat_head_stride = prm.stat_head_stride;
+    pp.stat_batch_stride = prm.stat_batch_stride;
+    pp.pre_tokens = pre;
+    pp.next_tokens = nxt;
+    pp.B = B;
+    pp.Nq = Nq;
+    pp.Nkv = Nkv;
+    pp.Sq = Sq;
+    pp.Skv = Skv;
+    pp.group = Nq / Nkv;
+    pp.sparse_mode = sparse_mode;
+    pp.tnd = tnd ? 1 : 0;
+    pp.head_grp = prm.head_grp;
+    pp.scale = scale;
+    int64_t n_pairs = 0;
+    if (tnd) {
+      pp.n_seq = prm.n_seq;
+      for (int i = 0; i < prm.n_seq; ++i) {
+        pp.seq_q_start[i] = prm.seq_q_start[i];
+        pp.seq_q_len[i] = prm.seq_q_len[i];
+        pp.seq_kv_start[i] = prm.seq_kv_start[i];
+        pp.seq_kv_len[i] = prm.seq_kv_len[i];
+        pp.seq_pair_start[i] = static_cast<int>(n_pairs);
+        n_pairs += ((prm.seq_q_len[i] + qbsa::kTile - 1) / qbsa::kTile + 1) / 2;
+      }
+      pp.seq_pair_start[prm.n_seq] = static_cast<int>(n_pairs);
+    } else {
+      pp.n_qtiles = (Sq + qbsa::kTile - 1) / qbsa::kTile;
+      pp.n_pair = (pp.n_qtiles + 1) / 2;
+      n_pairs = (int64_t)B * pp.n_pair;
+    }
+    pp.n_rank = static_cast<int>(n_pairs);
+    const int64_t n_pw = n_pairs * Nq;
+    if (n_pw == 0) return QBSA_OK;
+    if ((st = set_smem(qbsa::attn_pair_masked_kernel, qbsa::PairCfg::kSmemBytes)) != QBSA_OK) return st;
+    qbsa::attn_pair_masked_kernel<<<dim3(static_cast<unsigned>(n_pw)), qbsa::PairCfg::kThreads,
+                                    qbsa::PairCfg::kSmemBytes, s>>>(pp);
+    return check_launch("attn_pair_masked_kernel launch");
+  }
   if (block_mask) {
     prm.block_mask = block_mask;
     prm.mask_nkb = (Skv + qbsa::kTile - 1) / qbsa::kTile;
@@ -443,13 +500,13 @@ qbsa_status qbsa_quantize_qk(const void* x_bf16, int B, int N, int S, int D, int
 
 namespace {
 
-// Scratch of the V quantiser: ticket, per-head arrival counters, per-head column maxima.
-int64_t v_quant_scratch_words(int64_t H, int D) { return 1 + H + H * D; }
+// Scratch of the V quantiser: the per-head column maxima (float bits), zeroed before the first pass.
+int64_t v_quant_scratch_words(int64_t H, int D) { return H * D; }
 
 // Validates the V quantiser's arguments; on success fills the launch parameters (scratch
-// pointers excluded) and the persistent grid size.
+// pointer excluded).
 qbsa_status v_quant_setup(const void* v_bf16, int B, int N, int S, int D, uint8_t* codes, float* scales,
-                          qbsa::VQuantParams* prm, unsigned* grid) {
+                          qbsa::VQuantParams* prm) {
   if (!v_bf16 || !codes || !scales) return fail(QBSA_ERR_INVALID, "null pointer");
   if (B < 1 || N < 1 || S < 1 || D < 1) return fail(QBSA_ERR_INVALID, "B, N, S, D must be >= 1");
   if (D != 64 && D != 128 && D != 256) return fail(QBSA_ERR_UNSUPPORTED, "D must be 64, 128 or 256 (got %d)", D);
@@ -460,8 +517,7 @@ qbsa_status v_quant_setup(const void* v_bf16, int B, int N, int S, int D, uint8_
                                                                    : qbsa::VQuantCfg<256>::kRows;
   const int64_t H = (int64_t)B * N;
   const int64_t n_ch = (S + rows - 1) / rows;
-  if (2 * H * n_ch > 0xffffffffLL - 4 * 1024 * 1024 || H > 0x7fffffffLL)
-    return fail(QBSA_ERR_UNSUPPORTED, "too many (head, chunk) work items");
+  if (H * n_ch > 0x7fffffffLL) return fail(QBSA_ERR_UNSUPPORTED, "too many (head, chunk) blocks");
   memset(prm, 0, sizeof(*prm));
   prm->v = static_cast<const __nv_bfloat16*>(v_bf16);
   prm->codes = codes;
@@ -469,21 +525,17 @@ qbsa_status v_quant_setup(const void* v_bf16, int B, int N, int S, int D, uint8_
   prm->H = static_cast<int>(H);
   prm->S = S;
   prm->n_ch = static_cast<int>(n_ch);
-  prm->total = static_cast<unsigned int>(2 * H * n_ch);
-  int dev = 0, sms = 0, per_sm = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (e == cudaSuccess) {
-    e = D == 64 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, qbsa::v_quant_kernel<64>, qbsa::kQuantThreads, 0)
-        : D == 128 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, qbsa::v_quant_kernel<128>, qbsa::kQuantThreads, 0)
-                   : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, qbsa::v_quant_kernel<256>, qbsa::kQuantThreads, 0);
-  }
-  if (e != cudaSuccess) return cuda_fail(e, "querying the SM count / occupancy");
-  *grid = static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>((int64_t)sms * std::max(per_sm, 1), prm->total)));
   return QBSA_OK;
 }
 
-qbsa_status v_quant_launch(const qbsa::VQuantParams& prm, int D, unsigned grid, cudaStream_t st) {
+// Both passes, queued on `st` (prm.amax must already be zeroed on `st`).
+qbsa_status v_quant_launch(const qbsa::VQuantParams& prm, int D, cudaStream_t st) {
+  const unsigned grid = static_cast<unsigned>((int64_t)prm.H * prm.n_ch);
+  if (D == 64) qbsa::v_colmax_kernel<64><<<grid, qbsa::kQuantThreads, 0, st>>>(prm);
+  else if (D == 128) qbsa::v_colmax_kernel<128><<<grid, qbsa::kQuantThreads, 0, st>>>(prm);
+  else qbsa::v_colmax_kernel<256><<<grid, qbsa::kQuantThreads, 0, st>>>(prm);
+  qbsa_status r = check_launch("v_colmax_kernel launch");
+  if (r != QBSA_OK) return r;
   if (D == 64) qbsa::v_quant_kernel<64><<<grid, qbsa::kQuantThreads, 0, st>>>(prm);
   else if (D == 128) qbsa::v_quant_kernel<128><<<grid, qbsa::kQuantThreads, 0, st>>>(prm);
   else qbsa::v_quant_kernel<256><<<grid, qbsa::kQuantThreads, 0, st>>>(prm);
@@ -497,8 +549,7 @@ extern "C" {
 qbsa_status qbsa_quantize_v(const void* v_bf16, int B, int N, int S, int D, uint8_t* codes, float* scales,
                             void* stream) {
   qbsa::VQuantParams prm;
-  unsigned grid = 0;
-  qbsa_status st = v_quant_setup(v_bf16, B, N, S, D, codes, scales, &prm, &grid);
+  qbsa_status st = v_quant_setup(v_bf16, B, N, S, D, codes, scales, &prm);
   if (st != QBSA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const size_t bytes = static_cast<size_t>(v_quant_scratch_words(prm.H, D)) * sizeof(unsigned int);
@@ -510,11 +561,8 @@ qbsa_status qbsa_quantize_v(const void* v_bf16, int B, int N, int S, int D, uint
     cudaFreeAsync(scratch, s);
     return cuda_fail(e, "cudaMemsetAsync (V quantiser scratch)");
   }
-  unsigned int* w = static_cast<unsigned int*>(scratch);
-  prm.ticket = w;
-  prm.arrived = w + 1;
-  prm.amax = w + 1 + prm.H;
-  st = v_quant_launch(prm, D, grid, s);
+  prm.amax = static_cast<unsigned int*>(scratch);
+  st = v_quant_launch(prm, D, s);
   e = cudaFreeAsync(scratch, s);
   if (st != QBSA_OK) return st;
   if (e != cudaSuccess) return cuda_fail(e, "cudaFreeAsync (V quantiser scratch)");
@@ -531,8 +579,8 @@ qbsa_status qbsa_quantize_v(const void* v_bf16, int B, int N, int S, int D, uint
 // runs inside a custom allocator or a memory-pool callback, callers whose device heap is
 // fully reserved up front (a serving process that pre-plans every byte), or runtimes
 // that forbid cudaMalloc / cudaMallocAsync on their streams.  This entry point gives them
-// the same V quantiser with its scratch (ticket counter, per-head arrival counters and
-// per-head column maxima) in a fixed array that lives in the library's device image.
+// the same V quantiser with its scratch (the per-head column maxima) in a fixed array that
+// lives in the library's device image.
 
 namespace {
 
@@ -568,23 +616,20 @@ extern "C" {
 qbsa_status qbsa_quantize_v_noalloc(const void* v_bf16, int B, int N, int S, int D, uint8_t* codes, float* scales,
                                     void* stream) {
   qbsa::VQuantParams prm;
-  unsigned grid = 0;
-  qbsa_status st = v_quant_setup(v_bf16, B, N, S, D, codes, scales, &prm, &grid);
+  qbsa_status st = v_quant_setup(v_bf16, B, N, S, D, codes, scales, &prm);
   if (st != QBSA_OK) return st;
   const int64_t words = v_quant_scratch_words(prm.H, D);
   if (words > kNoAllocScratchWords)
     return fail(QBSA_ERR_UNSUPPORTED,
-                "qbsa_quantize_v_noalloc: B*N*(D+1)+1 = %lld scratch words exceed the fixed %lld (256 KiB); "
+                "qbsa_quantize_v_noalloc: B*N*D = %lld scratch words exceed the fixed %lld (256 KiB); "
                 "use qbsa_quantize_v", (long long)words, (long long)kNoAllocScratchWords);
   unsigned int* w = nullptr;
   if ((st = vq_scratch_address(&w)) != QBSA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaMemsetAsync(w, 0, static_cast<size_t>(words) * sizeof(unsigned int), s);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync (V quantiser scratch)");
-  prm.ticket = w;
-  prm.arrived = w + 1;
-  prm.amax = w + 1 + prm.H;
-  return v_quant_launch(prm, D, grid, s);
+  prm.amax = w;
+  return v_quant_launch(prm, D, s);
 }
 
 }  // extern "C"

@@ -52,7 +52,7 @@ def _run_and_compare(q, k, v, layout, Nq, scale, mode=0, pre=INF, nxt=INF, mask=
     (2, 2, 2, 129, 100, 128, 0, INF, INF, "BNSD"),
     (1, 1, 1, 1, 700, 64, 3, INF, INF, "BNSD"),
     (1, 3, 1, 1000, 1000, 128, 2, INF, INF, "BNSD"),
-    # two-tile kernel with per-tile K ranges
+    # masked two-tile kernel (per-tile K ranges)
     (1, 2, 1, 600, 600, 128, 0, 0, 0, "BNSD"),         # diagonal-only band: one K tile per query tile
     (1, 2, 2, 1000, 300, 128, 3, INF, INF, "BSND"),    # most rows have no key
     (2, 3, 1, 257, 1029, 128, 2, INF, INF, "BNSD"),    # top-left causal with S_kv > S_q
@@ -210,7 +210,7 @@ def _growing_k(k, Skv, factor=3.0):
     (1, 2, 2, 256, 680, 128, 0, "BNSD"),    # two-tile kernel, one pair per head, short last K tile
     (1, 3, 1, 650, 680, 128, 0, "BSND"),    # two-tile kernel, odd tile count
     (1, 2, 1, 300, 680, 64, 0, "BNSD"),     # one-tile kernel (D = 64)
-    (1, 2, 1, 300, 680, 128, 3, "BNSD"),    # two-tile kernel, causal (bottom-right): unequal K ranges
+    (1, 2, 1, 300, 680, 128, 3, "BNSD"),    # masked two-tile kernel, causal (bottom-right): unequal K ranges
 ])
 def test_dense_lazy_rescale_growing_k(B, Nq, Nkv, Sq, Skv, D, mode, layout):
     """The rescale of O in TMEM (taken only when the running max grows by more than 2^8)

@@ -43,7 +43,7 @@ def test_quantize_v_noalloc_matches_allocating_entry_point():
 
 
 def test_quantize_v_noalloc_rejects_sizes_beyond_its_scratch():
-    """B*N*(D+1) + 1 words above the fixed 65536 is refused before anything is queued."""
+    """B*N*D words above the fixed 65536 is refused before anything is queued."""
     L = qb.lib()
     v = torch.zeros((1, 8, 128, 128), dtype=torch.bfloat16, device="cuda")
     codes = torch.zeros((1, 8, 128, 128), dtype=torch.uint8, device="cuda")
