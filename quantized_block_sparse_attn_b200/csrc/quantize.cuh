@@ -173,8 +173,8 @@ template <int D>
 struct VQuantCfg {
   static constexpr int kTPR = D / 8;                   // threads per row, 8 channels each
   static constexpr int kRPI = kQuantThreads / kTPR;    // rows per iteration of the CTA
-  static constexpr int kIters = 16;
-  static constexpr int kRows = kRPI * kIters;          // rows per chunk (256 at D = 128)
+  static constexpr int kIters = 8;
+  static constexpr int kRows = kRPI * kIters;          // rows per chunk (128 at D = 128: 32 KB)
 };
 
 struct VQuantParams {
@@ -229,7 +229,7 @@ __global__ void __launch_bounds__(kQuantThreads) v_colmax_kernel(VQuantParams p)
 }
 
 template <int D>
-__global__ void __launch_bounds__(kQuantThreads) v_quant_kernel(VQuantParams p) {
+__global__ void __launch_bounds__(kQuantThreads, 3) v_quant_kernel(VQuantParams p) {
   using C = VQuantCfg<D>;
   const int tid = threadIdx.x;
   const int cg = tid % C::kTPR;
