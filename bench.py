@@ -670,7 +670,9 @@ def quantize_line(device, stream, S, hbm_peak):
             "qk_frac_of_hbm": qk_bytes / (qk_ms / 1e3) / 1e9 / hbm_peak,
             "v_ms": v_ms, "v_gbs": v_bytes / (v_ms / 1e3) / 1e9,
             "v_frac_of_hbm": v_bytes / (v_ms / 1e3) / 1e9 / hbm_peak,
+            "v_moved_frac_of_hbm": (v_bytes + N * S * D * 2) / (v_ms / 1e3) / 1e9 / hbm_peak,
             "algorithmic_bytes": "bf16 read once + 8-bit codes and fp32 scales written once",
+            "v_moved_bytes": "V's column maxima span all of S, so its bf16 is read twice (maxima, then codes)",
             "kernels": "quantize_qk_kernel<128>, v_quant_kernel<128> (one pass over HBM, re-read from L2)"}
 
 
