@@ -395,6 +395,10 @@ def run_ours(args):
                          "kernel": "attn_qbsa_kernel", "algorithmic_bytes": alg_bytes,
                          "hbm_gbs_algorithmic": alg_bytes / (launch_ms / 1e3) / 1e9},
             "gpu_launches": args.steps, "clocks": clocks}
+    mean_ms = sum(per_ms) / len(per_ms)
+    line["step_stats"] = {"median_ms": statistics.median(per_ms), "min_ms": min(per_ms), "max_ms": max(per_ms),
+                          "cv": (statistics.pstdev(per_ms) / mean_ms) if len(per_ms) > 1 else 0.0,
+                          "rule": "coefficient of variation of the per-step device times below 0.05"}
 
     # ---------------------------------------------------------------- e2e through the public API, host buffers
     if not args.no_e2e:
