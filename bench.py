@@ -38,9 +38,9 @@ FP8_OVER_BF16 = 2.0  # nominal dense ratio (4.5 vs 2.25 PFLOP/s), applied to the
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one attn_qbsa_kernel launch from
 # one ncu capture at S=16384, keep 0.1; it holds only for the kernel sources it was taken on,
 # identified by their sha1.
-QBSA_NCU_TRAFFIC = {"sources": {"quantized_block_sparse_attn_b200/csrc/attn_qbsa.cuh": "5a21fd90ccb9d35f74b4398bc7764686c1cf59fe",
+QBSA_NCU_TRAFFIC = {"sources": {"quantized_block_sparse_attn_b200/csrc/attn_qbsa.cuh": "57ac69cc0f60dc779bf1ce860d9f5d522335c4ff",
                                 "quantized_block_sparse_attn_b200/csrc/ptx_sm100.cuh": "76287e5abe014dfeeab1944e7be8a2564b0e0057"},
-                    "seq": 16384, "keep": 0.1, "bytes": 459491584, "alg_bytes": 420147200}
+                    "seq": 16384, "keep": 0.1, "bytes": 460804864, "alg_bytes": 420147200}
 
 
 def qbsa_traffic(seq: int, keep: float, alg_bytes: int):

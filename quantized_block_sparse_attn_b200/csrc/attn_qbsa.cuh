@@ -19,7 +19,10 @@
 //               softmax whose weights p = 2^(z - R) use a power-of-two reference R
 //               re-set to ceil(running max) only when the max exceeds it by more than 8
 //               (exact power-of-two rescales of O and L, rare);
-//               P -> FP16 -> E4M3 into TMEM; epilogue O * v_scale / L -> bf16 staged
+//               P -> FP16 -> E4M3 into TMEM.  A last kept block that runs past S_kv
+//               (ragged S_kv) is handled by an out-of-line copy of the step that masks
+//               the keys beyond S_kv, so the main loop carries no masking code.
+//               Epilogue O * v_scale / L -> bf16 staged
 //               in the tile's Q buffer (free by then) and a second buffer, written by
 //               TMA stores.
 //   warp 8      TMA producer: Q of both tiles once; K and V tiles of the kept blocks
@@ -161,6 +164,76 @@ __device__ __forceinline__ int compact_mask_row_v16(const uint8_t* row, int n_kb
     count += __shfl_sync(0xffffffffu, incl, 31);
   }
   return count;
+}
+
+struct QbsaTailResult {
+  float m, ref;
+  int ok;
+};
+
+// The softmax step of a row's last kept block when that block runs past S_kv (only the last
+// can: the kept lists are ascending).  Out of line so that the main loop carries no code for
+// the masking; called by the whole warp, at most once per row.  Same arithmetic as the loop.
+__device__ __noinline__ QbsaTailResult qbsa_tail_block(uint32_t s_col, uint32_t o_col, uint32_t p_col,
+                                                       uint32_t bar_sfull, uint32_t bar_sfree, uint32_t bar_pvdone,
+                                                       uint32_t bar_pfull, int j, float cst, int valid, float m,
+                                                       float ref, volatile int* abort_flag) {
+  const int lane = threadIdx.x & 31;
+  const float kNegInf = -__int_as_float(0x7f800000);
+  QbsaTailResult r{m, ref, 0};
+  if (!warp_wait(bar_sfull, static_cast<uint32_t>(j) & 1, abort_flag)) return r;
+  tc_fence_after();
+  uint32_t sv[128];
+  tmem_ld128_wait(s_col, sv);
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(bar_sfree);
+  const bool pos = cst >= 0.f;
+  const uint32_t pad = pos ? 0x80000000u : 0x7fffffffu;  // keys past S_kv take no part in the max
+#pragma unroll
+  for (int x = 0; x < 128; ++x)
+    if (x >= valid) sv[x] = pad;
+  const float m_blk = __int2float_rn(pos ? imax128(sv) : imin128(sv)) * cst;
+  m = fmaxf(m, m_blk);
+  const bool upd = (ref == kNegInf) || (m > ref + 8.0f);
+  const float new_ref = upd ? ceilf(m) : ref;
+  const bool need = upd && (ref != kNegInf);
+  const int dexp = need ? static_cast<int>(ref - new_ref) : 0;
+  const float a = (dexp < -126) ? 0.f : __int_as_float((127 + dexp) << 23);
+  ref = new_ref;
+  const uint64_t cc = pack_f32x2(cst, cst);
+  const uint64_t nr = pack_f32x2(-ref, -ref);
+  uint32_t pk[32];
+#pragma unroll
+  for (int x = 0; x < 32; ++x) {
+    pk[x] = i2f_fma_exp2_e4m3x4(sv[4 * x], sv[4 * x + 1], sv[4 * x + 2], sv[4 * x + 3], cc, nr);
+    const int keep = min(max(valid - 4 * x, 0), 4);  // zero the weights of keys past S_kv
+    pk[x] &= (keep == 4) ? 0xffffffffu : ((1u << (8 * keep)) - 1u);
+  }
+  if (j > 0) {
+    if (!warp_wait(bar_pvdone, static_cast<uint32_t>(j - 1) & 1, abort_flag)) return r;
+    tc_fence_after();
+    if (__any_sync(0xffffffffu, need)) {
+      uint32_t rr[32];
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        tmem_ld32_wait(o_col + ch * 32, rr);
+#pragma unroll
+        for (int x = 0; x < 32; ++x) rr[x] = __float_as_uint(__uint_as_float(rr[x]) * a);
+        tmem_st32(o_col + ch * 32, rr);
+      }
+      tmem_st1(o_col + 128, __float_as_uint(__uint_as_float(tmem_ld1_wait(o_col + 128)) * a));
+    }
+  }
+  tmem_st32(p_col, pk);
+  tmem_st_wait();
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(bar_pfull);
+  r.m = m;
+  r.ref = ref;
+  r.ok = 1;
+  return r;
 }
 
 __global__ void __launch_bounds__(352, 1) attn_qbsa_kernel(const __grid_constant__ QbsaParams p) {
@@ -394,15 +467,16 @@ __global__ void __launch_bounds__(352, 1) attn_qbsa_kernel(const __grid_constant
 
     float m = kNegInf;    // running max, log2 domain
     float ref = kNegInf;  // power-of-two reference of the FP8 weights (an integer)
+    // a last kept block that runs past S_kv is taken out of line after the loop
+    const bool tail_last = nt > 0 && (p.Skv % kTile) != 0 && list[nt - 1] == p.nkb - 1;
+    const int n_main = nt - (tail_last ? 1 : 0);
     bool ok = true;
-    for (int j = 0; ok && j < nt; ++j) {
-      const int kb = kb_next;
+    for (int j = 0; ok && j < n_main; ++j) {
       const float cst = (sq * ks_next) * p.scale_log2;
       if (j + 1 < nt) {  // the next block's key scale, fetched while this block is processed
         kb_next = list[j + 1];
         ks_next = ks_row[kb_next];
       }
-      const int valid = min(kTile, p.Skv - kb * kTile);  // key columns inside S_kv
       ok = warp_wait(bar(C::kBarSFull + t), static_cast<uint32_t>(j) & 1, abort_flag);
       if (!ok) break;
       tc_fence_after();
@@ -414,12 +488,6 @@ __global__ void __launch_bounds__(352, 1) attn_qbsa_kernel(const __grid_constant
 
       // row max of z = t * c: max(t) * c for c >= 0, min(t) * c otherwise (c is uniform)
       const bool pos = cst >= 0.f;
-      if (valid < kTile) {  // tail block: keys past S_kv take no part
-        const uint32_t pad = pos ? 0x80000000u : 0x7fffffffu;
-#pragma unroll
-        for (int x = 0; x < 128; ++x)
-          if (x >= valid) sv[x] = pad;
-      }
       const float m_blk = __int2float_rn(pos ? imax128(sv) : imin128(sv)) * cst;
       m = fmaxf(m, m_blk);
       // power-of-two reference: re-set to ceil(m) once m exceeds it by more than 8, so
@@ -440,13 +508,6 @@ __global__ void __launch_bounds__(352, 1) attn_qbsa_kernel(const __grid_constant
 #pragma unroll
       for (int x = 0; x < 32; ++x)
         pk[x] = i2f_fma_exp2_e4m3x4(sv[4 * x], sv[4 * x + 1], sv[4 * x + 2], sv[4 * x + 3], cc, nr);
-      if (valid < kTile) {  // tail block: zero the weights of keys past S_kv whatever c is
-#pragma unroll
-        for (int x = 0; x < 32; ++x) {
-          const int keep = min(max(valid - 4 * x, 0), 4);
-          pk[x] &= (keep == 4) ? 0xffffffffu : ((1u << (8 * keep)) - 1u);
-        }
-      }
 
       // P_t and O_t are free once the previous block's P·V has retired
       if (j > 0) {
@@ -470,6 +531,15 @@ __global__ void __launch_bounds__(352, 1) attn_qbsa_kernel(const __grid_constant
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(C::kBarPFull + t));
+    }
+    if (ok && tail_last) {
+      const int kb = kb_next;  // list[nt - 1]
+      const QbsaTailResult r = qbsa_tail_block(s_col, o_col, p_col, bar(C::kBarSFull + t), bar(C::kBarSFree + t),
+                                               bar(C::kBarPVDone + t), bar(C::kBarPFull + t), nt - 1,
+                                               (sq * ks_next) * p.scale_log2, p.Skv - kb * kTile, m, ref, abort_flag);
+      m = r.m;
+      ref = r.ref;
+      ok = r.ok != 0;
     }
 
     // ------------------------------------------------------------ epilogue
