@@ -180,6 +180,16 @@ def qbsa_work(inp):
     return executed, dense_eq, bytes_
 
 
+def step_stats(per_ms):
+    """Median, extremes and coefficient of variation of per-step device times (ms); the
+    stability rule asks for a CV below 0.05."""
+    mean_ms = sum(per_ms) / len(per_ms)
+    return {"median_ms": statistics.median(per_ms), "min_ms": min(per_ms), "max_ms": max(per_ms),
+            "cv": (statistics.pstdev(per_ms) / mean_ms) if len(per_ms) > 1 else 0.0,
+            "stable": len(per_ms) < 2 or statistics.pstdev(per_ms) / mean_ms < 0.05,
+            "rule": "coefficient of variation of the per-step device times below 0.05"}
+
+
 def time_steps(fn, steps: int, warmup: int, stream, dist=None, sampler=None, flush=None):
     """Run fn warmup times, then time exactly `steps` calls with CUDA events on `stream`.
 
@@ -395,10 +405,7 @@ def run_ours(args):
                          "kernel": "attn_qbsa_kernel", "algorithmic_bytes": alg_bytes,
                          "hbm_gbs_algorithmic": alg_bytes / (launch_ms / 1e3) / 1e9},
             "gpu_launches": args.steps, "clocks": clocks}
-    mean_ms = sum(per_ms) / len(per_ms)
-    line["step_stats"] = {"median_ms": statistics.median(per_ms), "min_ms": min(per_ms), "max_ms": max(per_ms),
-                          "cv": (statistics.pstdev(per_ms) / mean_ms) if len(per_ms) > 1 else 0.0,
-                          "rule": "coefficient of variation of the per-step device times below 0.05"}
+    line["step_stats"] = step_stats(per_ms)
 
     # ---------------------------------------------------------------- e2e through the public API, host buffers
     if not args.no_e2e:

@@ -43,3 +43,35 @@ def test_algorithmic_work_of_the_workload():
     assert dense_eq == 4.0 * 128 * 65536 * 65536 * 40
     # Q, K, V bytes read once (int8 / e4m3), bf16 output, mask and scales
     assert nbytes == 3 * 40 * 65536 * 128 + 2 * 40 * 65536 * 128 + 40 * 512 * 512 + 4 * (2 * 40 * 512 + 40 * 128)
+
+
+def test_step_stats_median_and_cv():
+    bench = _bench()
+    st = bench.step_stats([1.0, 1.0, 1.0, 1.0])
+    assert st["median_ms"] == 1.0 and st["cv"] == 0.0 and st["stable"]
+    st = bench.step_stats([1.0, 2.0, 3.0])  # pstdev sqrt(2/3), mean 2
+    assert st["median_ms"] == 2.0 and st["min_ms"] == 1.0 and st["max_ms"] == 3.0
+    assert abs(st["cv"] - (2.0 / 3.0) ** 0.5 / 2.0) < 1e-12 and not st["stable"]
+    assert bench.step_stats([5.0])["cv"] == 0.0
+
+
+def test_reference_arm_prints_the_contract_line():
+    """`bench.py --impl reference` times the CPU oracle (no GPU needed) and prints one JSON
+    line with the reference arm's keys."""
+    import json
+    import subprocess
+    import sys
+    res = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+                          "--warmup", "0"], capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert res.returncode == 0, res.stderr[-2000:]
+    lines = [l for l in res.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["steps"] == 1 and d["warmup"] == 0 and d["n_gpus"] == 1
+    assert d["metric"] == bench_metric() and d["unit"] == "TFLOP/s" and d["value"] > 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def bench_metric():
+    return _bench().METRIC
