@@ -137,6 +137,19 @@ def _block_scores(qi, k8, qs_b, ks_b, scale, c0, c1):
     return t.astype(np.float64) * (float(qs_b) * float(ks_b) * scale)
 
 
+def _log2_scale_f32(scale):
+    """scale·log2(e) as the kernel's host code forms it: both factors in f32, one f32 product."""
+    return np.float32(np.float32(scale) * np.float32(LOG2E))
+
+
+def _block_products_f32(qi, k8, qs_b, ks_b, sl, c0, c1):
+    """For the kernel's reading: t and c = f32(f32(s_q·s_k)·sl) for one kept key block, and
+    the exact products t·c (|t| < 2^21 times a 24-bit c is exact in fp64)."""
+    t = qi @ k8[c0:c1].astype(np.int64).T
+    c = np.float32(np.float32(np.float32(qs_b) * np.float32(ks_b)) * sl)
+    return t.astype(np.float64) * float(c)
+
+
 def _head_plain(q8, k8, qs, ks, v8f, vs, mask_rows, scale, qbs, round_p=True):
     """Plain online-softmax reading for one (b, h): running max moved and l, acc rescaled
     at every kept block; weights E4M3(FP16(e^(s - m))) against that running max."""
@@ -169,8 +182,15 @@ def _head_plain(q8, k8, qs, ks, v8f, vs, mask_rows, scale, qbs, round_p=True):
 
 def _head_pow2ref(q8, k8, qs, ks, v8f, vs, mask_rows, scale, qbs, round_p=True):
     """Kernel's reading for one (b, h): weights E4M3(FP16(2^(z - R))) against a lazily moved
-    power-of-two reference R (re-set to ceil(m) only when m passes R + REF_SLACK)."""
+    power-of-two reference R (re-set to ceil(m) only when m passes R + REF_SLACK).
+
+    The FP16 and E4M3 codes of each weight are decided on z, so z is formed in the kernel's
+    precision: c = s_q·s_k·scale·log2(e) in f32 (as the kernel forms it), the block maximum
+    as f32(t_max·c), and z − R = f32(t·c − R) with one rounding (a fused multiply-add).
+    2^(z − R) itself is exact here (the kernel's ex2.approx differs from it only in the last
+    bits of f32)."""
     skv, D = k8.shape[0], v8f.shape[1]
+    sl = _log2_scale_f32(scale)
     outs, mxs, sms = [], [], []
     for qb in qbs:
         r0, r1 = qb * BLK, min(q8.shape[0], (qb + 1) * BLK)
@@ -182,14 +202,14 @@ def _head_pow2ref(q8, k8, qs, ks, v8f, vs, mask_rows, scale, qbs, round_p=True):
         acc = np.zeros((rows, D))
         for kb in np.nonzero(mask_rows[qb])[0]:                               # ascending
             c0, c1 = kb * BLK, min(skv, (kb + 1) * BLK)
-            z = _block_scores(qi, k8, qs[qb], ks[kb], scale, c0, c1) * LOG2E
-            m = np.maximum(m, z.max(axis=1))
+            tc = _block_products_f32(qi, k8, qs[qb], ks[kb], sl, c0, c1)
+            m = np.maximum(m, tc.max(axis=1).astype(np.float32).astype(np.float64))
             upd = np.isneginf(ref) | (m > ref + REF_SLACK)
             new_ref = np.where(upd, np.ceil(m), ref)
             unset = np.isneginf(ref)
             alpha = np.where(unset, 0.0, np.exp2(np.where(unset, 0.0, ref) - new_ref))  # exact powers of two
             l, acc, ref = l * alpha, acc * alpha[:, None], new_ref
-            p = np.exp2(z - ref[:, None])
+            p = np.exp2((tc - ref[:, None]).astype(np.float32).astype(np.float64))
             if round_p:
                 p = _fp8_weights(p)
             l = l + p.sum(axis=1)
@@ -272,20 +292,20 @@ def _loops(q8, k8, q_scale, k_scale, v8, v_scale, block_mask, scale, pow2ref):
                     if not block_mask[b, h, qb, kb]:
                         continue
                     cols = range(kb * BLK, min(Skv, (kb + 1) * BLK))
-                    s = []
-                    for j in cols:
-                        t = sum(int(q8[b, h, i, c]) * int(k8[b, g, j, c]) for c in range(D))
-                        s.append(t * (float(q_scale[b, h, qb]) * float(k_scale[b, g, kb]) * scale))
+                    ts = [sum(int(q8[b, h, i, c]) * int(k8[b, g, j, c]) for c in range(D)) for j in cols]
+                    s = [t * (float(q_scale[b, h, qb]) * float(k_scale[b, g, kb]) * scale) for t in ts]
                     if pow2ref:
-                        z = [x * LOG2E for x in s]
-                        m = max(m, max(z))
+                        # the kernel's precision: f32 c, f32 block max, z - R rounded once to f32
+                        cf = float(np.float32(np.float32(np.float32(q_scale[b, h, qb]) * np.float32(k_scale[b, g, kb]))
+                                              * np.float32(np.float32(scale) * np.float32(LOG2E))))
+                        m = max(m, max(float(np.float32(t * cf)) for t in ts))
                         if ref == -math.inf or m > ref + REF_SLACK:
                             new_ref = math.ceil(m)
                             alpha = 0.0 if ref == -math.inf else 2.0 ** (ref - new_ref)
                             l *= alpha
                             acc = [a * alpha for a in acc]
                             ref = new_ref
-                        ws = [2.0 ** (zj - ref) for zj in z]
+                        ws = [2.0 ** float(np.float32(t * cf - ref)) for t in ts]
                     else:
                         m_new = max(m, max(s))
                         alpha = 0.0 if m == -math.inf else math.exp(m - m_new)

@@ -68,6 +68,65 @@ def test_qbsa_unequal_tile_pairs(sign):
     check_qbsa(got, gmax, gsum, q8, k8, qs, ks, v8, vs, bm, scale, tag=f"unequal pairs sign {sign}:")
 
 
+def _reference_moves(q8, qs, k8, ks, bm, scale, group):
+    """Per (b, h, query row), the kept blocks at which the running max of z = t·c (log2 units)
+    passes the power-of-two reference by more than 8 after the row's first block, i.e. where
+    the kernel rescales O and L.  Returns (count of such events, events at a ragged last block)."""
+    B, Nq, Sq, _ = q8.shape
+    Skv = k8.shape[2]
+    nkb = -(-Skv // 128)
+    ragged = Skv % 128 != 0
+    events = tail_events = 0
+    for b in range(B):
+        for h in range(Nq):
+            g = h // group
+            t_all = q8[b, h].astype(np.int64) @ k8[b, g].astype(np.int64).T  # [Sq, Skv]
+            for qb_ in range(-(-Sq // 128)):
+                rows = slice(qb_ * 128, min(Sq, (qb_ + 1) * 128))
+                m = np.full(rows.stop - rows.start, -np.inf)
+                ref = np.full_like(m, -np.inf)
+                for kb in np.nonzero(bm[b, h, qb_])[0]:
+                    cols = slice(kb * 128, min(Skv, (kb + 1) * 128))
+                    c = qs[b, h, qb_] * ks[b, g, kb] * scale * np.log2(np.e)
+                    z = t_all[rows, cols] * c
+                    m = np.maximum(m, z.max(axis=1))
+                    move = np.isfinite(ref) & (m > ref + 8)
+                    events += int(move.sum())
+                    if ragged and kb == nkb - 1:
+                        tail_events += int(move.sum())
+                    ref = np.where(~np.isfinite(ref) | (m > ref + 8), np.ceil(m), ref)
+    return events, tail_events
+
+
+@pytest.mark.parametrize("sign", [1.0, -1.0])
+def test_qbsa_growing_keys_rescale_and_ragged_tail(sign):
+    """Key blocks grow in magnitude (block j of K times 1 + 2 j before quantisation), so the
+    running max of every row passes the power-of-two reference by more than 8 several times
+    and O and L are rescaled in TMEM, also inside the out-of-line step of the ragged last key
+    block; B = 2, GQA 4:2, ragged on both axes, some blocks dropped.  A negative scale runs
+    the same through the row-minimum path."""
+    from workloads import bf16_bits_from_f32, bf16_bits_to_f32
+    B, Nq, Nkv, Sq, Skv, D = 2, 4, 2, 300, 1000, 128
+    q = iid_normal_bf16(31, 0, B, Nq, Sq, D)
+    kf = bf16_bits_to_f32(iid_normal_bf16(31, 1, B, Nkv, Skv, D)).copy()
+    for j in range(-(-Skv // 128)):
+        kf[:, :, j * 128:(j + 1) * 128] *= 1.0 + 2.0 * j
+    k = bf16_bits_from_f32(kf)
+    v = iid_normal_bf16(31, 2, B, Nkv, Skv, D)
+    q8, qs, k8, ks, v8, vs = _quantized(q, k, v)
+    nqb, nkb = -(-Sq // 128), -(-Skv // 128)
+    bm = np.ones((B, Nq, nqb, nkb), dtype=np.uint8)
+    bm[0, 1, :, 3] = 0
+    bm[1, 2, 0, 1:5] = 0
+    bm[1, 3, 2, :nkb - 1] = 0   # a row whose only block is the ragged one
+    scale = sign * D ** -0.5
+    events, tail_events = _reference_moves(q8, qs, k8, ks, bm, scale, Nq // Nkv)
+    assert events > 1000 and tail_events > 100, (events, tail_events)
+    got, gmax, gsum = _run(q8, qs, k8, ks, v8, vs, bm, scale)
+    check_qbsa(got, gmax, gsum, q8, k8, qs, ks, v8, vs, bm, scale,
+               tag=f"growing keys sign {sign} ({events} reference moves, {tail_events} in the ragged block):")
+
+
 @pytest.mark.parametrize("sign", [1.0, -1.0])
 def test_qbsa_more_units_than_sms(sign):
     """More (head, query-block pair) units than SMs, so the grid runs in several waves and
