@@ -35,6 +35,8 @@ def _run_and_compare(q, k, v, layout, Nq, scale, mode=0, pre=INF, nxt=INF, mask=
                                               actual_seq_kvlen=ck, q_rows=q_rows, heads=heads)
     mx, mn = compare_out(host_f64(out), ref, DENSE_MAX_ABS, DENSE_MEAN_ABS)
     compare_stats(smax.cpu().numpy(), ssum.cpu().numpy(), rmax, rsum)
+    print(f"{layout} Sq={q.shape[2] if layout == 'BNSD' else q.shape[1] if layout == 'BSND' else q.shape[0]} "
+          f"mode {mode}: max abs err {mx:.3e}, mean abs err {mn:.3e}")
     return mx, mn
 
 
