@@ -431,7 +431,8 @@ def run_ours(args):
         e2e_s = max_over_ranks((time.perf_counter() - t0) / e2e_steps, dist)
         line["e2e"] = {"value": world * executed / e2e_s / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                        "d2h_bytes_per_step": d2h, "ms_per_step": 1e3 * e2e_s,
-                       "note": "host pinned int8/e4m3/fp32 inputs copied in, bf16 output copied out, every step"}
+                       "note": "through the C ABI's qbsa_fwd_host: host pinned int8/e4m3/fp32 inputs copied in, "
+                               "bf16 output copied out, every step"}
 
     # ---------------------------------------------------------------- CPU oracle sample (rank 0, N=1)
     if rank == 0 and world == 1 and not args.no_cpu:

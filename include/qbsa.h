@@ -150,6 +150,26 @@ qbsa_status qbsa_fwd(const int8_t* q_i8, const int8_t* k_i8, const float* q_bloc
                      float* softmax_sum, void* stream);
 
 /*
+ * qbsa_fwd_host -- qbsa_fwd on HOST buffers: the same operation, arguments, layouts and
+ * outputs, but every data pointer (inputs, attention_out, the optional softmax_max /
+ * softmax_sum) is host memory.  Page-locked memory lets the copies overlap the kernel;
+ * pageable memory works, with the copies staged by the driver.
+ * The work is split into about n_chunks independent (batch, kv-head range) chunks (n_chunks
+ * >= 1; a chunk holds whole GQA groups).  Chunk c + 1's inputs are copied to the device on
+ * one library-owned stream while chunk c runs on `stream` and chunk c - 1's outputs return
+ * on another, ordered by events.  Device buffers come from a stream-ordered memory pool the
+ * library keeps per device (its memory is kept for later calls, never freed before the
+ * process exits).  The call returns after the results are in host memory; the host buffers
+ * must not be touched by other threads during the call.  Errors as qbsa_fwd, plus
+ * QBSA_ERR_INVALID for n_chunks < 1; a CUDA error during the copies returns QBSA_ERR_CUDA
+ * (the outputs are then unspecified).
+ */
+qbsa_status qbsa_fwd_host(const int8_t* q_i8, const int8_t* k_i8, const float* q_block_scale,
+                          const float* k_block_scale, const uint8_t* v_fp8, const float* v_channel_scale,
+                          const uint8_t* block_mask, int B, int Nq, int Nkv, int Sq, int Skv, int D, float scale,
+                          void* attention_out, float* softmax_max, float* softmax_sum, int n_chunks, void* stream);
+
+/*
  * qbsa_quantize_qk -- per-128-token-block symmetric INT8 quantisation of Q or K
  * ([QBSA] "EagleQBSA量化叠加稀疏方案设计"): for each (b, h, block) a = max|x| (fp32),
  * s = a/127 (1 if a = 0), codes = rint_half_even(x/s) clamped to [-127, 127].
@@ -278,8 +298,9 @@ qbsa_status qbsa_check(void* stream);
 /* Thread-local description of the last non-OK status returned on this thread. */
 const char* qbsa_last_error(void);
 
-/* Library ABI version (major * 100 + minor): 102 (1.01 added qbsa_block_mean, qbsa_block_topk,
- * qbsa_wait_selftest; 1.02 added qbsa_block_topk_keep). */
+/* Library ABI version (major * 100 + minor): 103 (1.01 added qbsa_block_mean, qbsa_block_topk,
+ * qbsa_wait_selftest; 1.02 qbsa_block_topk_keep and qbsa_quantize_v_noalloc; 1.03
+ * qbsa_fwd_host). */
 int qbsa_version(void);
 
 #ifdef __cplusplus

@@ -28,6 +28,7 @@ SIGNATURES = {
     "attn_fwd": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _I, _P, _I, _F, _F, _I, _I64, _I64,
                       _P, _P, _P, _P, _P, _P]),
     "qbsa_fwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P]),
+    "qbsa_fwd_host": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _I, _P]),
     "bsa_fwd": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P]),
     "qbsa_quantize_qk": (_I, [_P, _I, _I, _I, _I, _P, _P, _P]),
     "qbsa_quantize_v": (_I, [_P, _I, _I, _I, _I, _P, _P, _P]),
@@ -209,72 +210,22 @@ def bsa_fwd(q, k, v, block_mask, scale: float, *, out=None, softmax_max=None, so
     return out, softmax_max, softmax_sum
 
 
-_COPY_STREAMS = {}
-
-
-def _copy_streams(dev):
-    """Two side streams per device: host-to-device and device-to-host copies."""
-    import torch
-    key = dev.index if dev.index is not None else torch.cuda.current_device()
-    if key not in _COPY_STREAMS:
-        _COPY_STREAMS[key] = (torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev))
-    return _COPY_STREAMS[key]
-
-
 def _qbsa_fwd_host(q_i8, k_i8, q_scale, k_scale, v_fp8, v_scale, block_mask, scale, dsts, return_stats, dev,
                    n_chunks):
-    """qbsa_fwd on host tensors, pipelined over independent (batch, head) chunks: chunk c + 1's
-    inputs cross PCIe on one stream while chunk c runs on the current stream and chunk c - 1's
-    outputs return on another, so transfers in both directions overlap the kernel."""
+    """qbsa_fwd on host tensors through the library's qbsa_fwd_host (chunked copies that
+    overlap the kernel, done natively); returns host tensors (the caller's, or new pinned ones)."""
     import torch
     B, Nq, Sq, D = q_i8.shape
     Nkv, Skv = k_i8.shape[1], k_i8.shape[2]
-    if Nkv < 1 or Nq % Nkv != 0:
-        raise QbsaError(1, f"Nq ({Nq}) must be a multiple of Nkv ({Nkv})")
-    group = Nq // Nkv
-    pin = lambda t: t if t.is_pinned() else t.pin_memory()
-    hq = [pin(t.contiguous()) for t in (q_i8, k_i8, q_scale, k_scale, v_fp8, v_scale, block_mask)]
-    dq = [torch.empty(t.shape, dtype=t.dtype, device=dev) for t in hq]
-    d_out = torch.empty((B, Nq, Sq, D), dtype=torch.bfloat16, device=dev)
-    d_max = torch.empty((B, Nq, Sq), dtype=torch.float32, device=dev) if return_stats else None
-    d_sum = torch.empty((B, Nq, Sq), dtype=torch.float32, device=dev) if return_stats else None
-    h_out = dsts[0] if dsts[0] is not None else torch.empty(d_out.shape, dtype=d_out.dtype, pin_memory=True)
+    hq = [t.contiguous() for t in (q_i8, k_i8, q_scale, k_scale, v_fp8, v_scale, block_mask)]
+    h_out = dsts[0] if dsts[0] is not None else torch.empty((B, Nq, Sq, D), dtype=torch.bfloat16, pin_memory=True)
     h_max = h_sum = None
     if return_stats:
-        h_max = dsts[1] if dsts[1] is not None else torch.empty(d_max.shape, dtype=torch.float32, pin_memory=True)
-        h_sum = dsts[2] if dsts[2] is not None else torch.empty(d_sum.shape, dtype=torch.float32, pin_memory=True)
-    per_b = max(1, min(Nkv, -(-n_chunks // B)))
-    chunks = []
-    for b in range(B):
-        for c in range(per_b):
-            g0, g1 = c * Nkv // per_b, (c + 1) * Nkv // per_b
-            if g1 > g0:
-                chunks.append((b, g0, g1))
-    s_in, s_out = _copy_streams(dev)
-    s_comp = torch.cuda.current_stream(dev)
-    L = lib()
-    for b, g0, g1 in chunks:
-        h0, h1 = g0 * group, g1 * group
-        q_sl = (slice(b, b + 1), slice(h0, h1))
-        kv_sl = (slice(b, b + 1), slice(g0, g1))
-        sls = [q_sl, kv_sl, q_sl, kv_sl, kv_sl, kv_sl, q_sl]  # q8, k8, qs, ks, v8, vs, mask
-        with torch.cuda.stream(s_in):
-            for d, h, sl in zip(dq, hq, sls):
-                d[sl].copy_(h[sl], non_blocking=True)
-        s_comp.wait_stream(s_in)
-        dv = [d[sl] for d, sl in zip(dq, sls)]
-        o = d_out[q_sl]
-        mx = d_max[q_sl] if return_stats else None
-        sm = d_sum[q_sl] if return_stats else None
-        _ck(L.qbsa_fwd(_ptr(dv[0]), _ptr(dv[1]), _ptr(dv[2]), _ptr(dv[3]), _ptr(dv[4]), _ptr(dv[5]), _ptr(dv[6]), 1,
-                       h1 - h0, g1 - g0, Sq, Skv, D, scale, _ptr(o), _ptr(mx), _ptr(sm), _stream(dev)))
-        s_out.wait_stream(s_comp)
-        with torch.cuda.stream(s_out):
-            h_out[q_sl].copy_(o, non_blocking=True)
-            if return_stats:
-                h_max[q_sl].copy_(mx, non_blocking=True)
-                h_sum[q_sl].copy_(sm, non_blocking=True)
-    s_out.synchronize()
+        h_max = dsts[1] if dsts[1] is not None else torch.empty((B, Nq, Sq), dtype=torch.float32, pin_memory=True)
+        h_sum = dsts[2] if dsts[2] is not None else torch.empty((B, Nq, Sq), dtype=torch.float32, pin_memory=True)
+    with torch.cuda.device(dev):
+        _ck(lib().qbsa_fwd_host(*[_ptr(t) for t in hq], B, Nq, Nkv, Sq, Skv, D, scale, _ptr(h_out), _ptr(h_max),
+                                _ptr(h_sum), n_chunks, _stream(dev)))
     return h_out, h_max, h_sum
 
 
@@ -282,9 +233,10 @@ def qbsa_fwd(q_i8, k_i8, q_scale, k_scale, v_fp8, v_scale, block_mask, scale: fl
              softmax_max=None, softmax_sum=None, return_stats: bool = True, device=None, host_chunks: int = 8):
     """Quantized block-sparse attention forward (BNSD, D = 128).  Returns (out, max, sum).
 
-    Device tensors run as one launch on the current stream.  Host tensors are copied in and
-    the results copied out in `host_chunks` (batch, head) chunks whose transfers overlap the
-    kernel; the host results are pinned tensors (or the caller's `out` / stats tensors)."""
+    Device tensors run as one launch on the current stream.  Host tensors go through the
+    library's qbsa_fwd_host, which copies them in and the results out in about `host_chunks`
+    (batch, kv-head) chunks whose transfers overlap the kernel (page-locked tensors overlap
+    best); the host results are pinned tensors (or the caller's `out` / stats tensors)."""
     import torch
     host = not q_i8.is_cuda
     dev = torch.device(device or (q_i8.device if q_i8.is_cuda else "cuda:0"))

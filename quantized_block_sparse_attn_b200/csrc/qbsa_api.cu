@@ -126,7 +126,7 @@ qbsa_status launch_dense(qbsa::DenseParams& prm, int64_t n_work, cudaStream_t st
 
 extern "C" {
 
-int qbsa_version(void) { return 102; }
+int qbsa_version(void) { return 103; }
 
 const char* qbsa_last_error(void) { return g_last_error.c_str(); }
 
@@ -411,6 +411,23 @@ qbsa_status bsa_fwd(const void* q, const void* k, const void* v, const uint8_t* 
 // qbsa_fwd
 // ------------------------------------------------------------------------------
 
+}  // extern "C"
+
+// The shape checks qbsa_fwd and qbsa_fwd_host share.
+static qbsa_status qbsa_shape_check(int B, int Nq, int Nkv, int Sq, int Skv, int D, float scale) {
+  if (B < 1 || Nq < 1 || Nkv < 1 || Sq < 0 || Skv < 0) return fail(QBSA_ERR_INVALID, "B, Nq, Nkv >= 1 and Sq, Skv >= 0");
+  if (Nq % Nkv != 0) return fail(QBSA_ERR_INVALID, "Nq (%d) must be a multiple of Nkv (%d)", Nq, Nkv);
+  if (D != 128) return fail(QBSA_ERR_UNSUPPORTED, "qbsa_fwd supports D = 128 (got %d)", D);
+  if (!std::isfinite(scale)) return fail(QBSA_ERR_INVALID, "scale must be finite");
+  if (Sq > kMaxLen || Skv > kMaxLen) return fail(QBSA_ERR_UNSUPPORTED, "sequence length above %lld", (long long)kMaxLen);
+  const int nkb = (Skv + 127) / 128;
+  if (nkb > qbsa::kQbsaMaxKBlocks)
+    return fail(QBSA_ERR_UNSUPPORTED, "ceil(Skv/128) = %d exceeds %d", nkb, qbsa::kQbsaMaxKBlocks);
+  return QBSA_OK;
+}
+
+extern "C" {
+
 qbsa_status qbsa_fwd(const int8_t* q_i8, const int8_t* k_i8, const float* q_block_scale, const float* k_block_scale,
                      const uint8_t* v_fp8, const float* v_channel_scale, const uint8_t* block_mask, int B, int Nq,
                      int Nkv, int Sq, int Skv, int D, float scale, void* attention_out, float* softmax_max,
@@ -420,14 +437,11 @@ qbsa_status qbsa_fwd(const int8_t* q_i8, const int8_t* k_i8, const float* q_bloc
     return fail(QBSA_ERR_INVALID, "all tensor arguments except the softmax statistics must be non-null");
   if (!aligned16(q_i8) || !aligned16(k_i8) || !aligned16(v_fp8) || !aligned16(attention_out))
     return fail(QBSA_ERR_INVALID, "q_i8, k_i8, v_fp8 and attention_out must be 16-byte aligned");
-  if (B < 1 || Nq < 1 || Nkv < 1 || Sq < 0 || Skv < 0) return fail(QBSA_ERR_INVALID, "B, Nq, Nkv >= 1 and Sq, Skv >= 0");
-  if (Nq % Nkv != 0) return fail(QBSA_ERR_INVALID, "Nq (%d) must be a multiple of Nkv (%d)", Nq, Nkv);
-  if (D != 128) return fail(QBSA_ERR_UNSUPPORTED, "qbsa_fwd supports D = 128 (got %d)", D);
-  if (!std::isfinite(scale)) return fail(QBSA_ERR_INVALID, "scale must be finite");
-  if (Sq > kMaxLen || Skv > kMaxLen) return fail(QBSA_ERR_UNSUPPORTED, "sequence length above %lld", (long long)kMaxLen);
+  {
+    const qbsa_status sc = qbsa_shape_check(B, Nq, Nkv, Sq, Skv, D, scale);
+    if (sc != QBSA_OK) return sc;
+  }
   const int nqb = (Sq + 127) / 128, nkb = (Skv + 127) / 128;
-  if (nkb > qbsa::kQbsaMaxKBlocks)
-    return fail(QBSA_ERR_UNSUPPORTED, "ceil(Skv/128) = %d exceeds %d", nkb, qbsa::kQbsaMaxKBlocks);
   if (Sq == 0) return QBSA_OK;
 
   qbsa::QbsaParams prm;
@@ -756,6 +770,176 @@ qbsa_status qbsa_check(void* stream) {
     cudaMemcpyToSymbol(qbsa::g_device_error, &zero, sizeof(zero));
     return fail(QBSA_ERR_TIMEOUT, "a kernel wait exceeded its time limit (device error word %u)", word);
   }
+  return QBSA_OK;
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------------------------
+// qbsa_fwd on host buffers: chunked copies that overlap the kernel
+// ------------------------------------------------------------------------------
+//
+// Per device the library keeps two non-blocking copy streams (host -> device, device ->
+// host) and a stream-ordered memory pool whose memory is kept between calls, so that a
+// call's device buffers cost no fresh allocation after the first call of that size.
+
+namespace {
+
+struct HostPathState {
+  bool ready = false;
+  cudaStream_t s_in = nullptr;
+  cudaStream_t s_out = nullptr;
+  cudaMemPool_t pool = nullptr;
+};
+
+constexpr int kHostPathDevices = 64;
+std::mutex g_host_path_mu;
+HostPathState g_host_path[kHostPathDevices];
+
+qbsa_status host_path_state(HostPathState** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kHostPathDevices) return fail(QBSA_ERR_UNSUPPORTED, "device ordinal %d", dev);
+  std::lock_guard<std::mutex> lock(g_host_path_mu);
+  HostPathState& st = g_host_path[dev];
+  if (!st.ready) {
+    if ((e = cudaStreamCreateWithFlags(&st.s_in, cudaStreamNonBlocking)) != cudaSuccess)
+      return cuda_fail(e, "cudaStreamCreateWithFlags (copy-in stream)");
+    if ((e = cudaStreamCreateWithFlags(&st.s_out, cudaStreamNonBlocking)) != cudaSuccess)
+      return cuda_fail(e, "cudaStreamCreateWithFlags (copy-out stream)");
+    cudaMemPoolProps props;
+    memset(&props, 0, sizeof(props));
+    props.allocType = cudaMemAllocationTypePinned;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    if ((e = cudaMemPoolCreate(&st.pool, &props)) != cudaSuccess) return cuda_fail(e, "cudaMemPoolCreate");
+    uint64_t keep = ~0ull;
+    if ((e = cudaMemPoolSetAttribute(st.pool, cudaMemPoolAttrReleaseThreshold, &keep)) != cudaSuccess)
+      return cuda_fail(e, "cudaMemPoolSetAttribute");
+    st.ready = true;
+  }
+  *out = &st;
+  return QBSA_OK;
+}
+
+size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+
+}  // namespace
+
+extern "C" {
+
+qbsa_status qbsa_fwd_host(const int8_t* q_i8, const int8_t* k_i8, const float* q_block_scale,
+                          const float* k_block_scale, const uint8_t* v_fp8, const float* v_channel_scale,
+                          const uint8_t* block_mask, int B, int Nq, int Nkv, int Sq, int Skv, int D, float scale,
+                          void* attention_out, float* softmax_max, float* softmax_sum, int n_chunks, void* stream) {
+  if (!q_i8 || !k_i8 || !q_block_scale || !k_block_scale || !v_fp8 || !v_channel_scale || !block_mask ||
+      !attention_out)
+    return fail(QBSA_ERR_INVALID, "all tensor arguments except the softmax statistics must be non-null");
+  if (n_chunks < 1) return fail(QBSA_ERR_INVALID, "n_chunks must be >= 1 (got %d)", n_chunks);
+  {
+    const qbsa_status sc = qbsa_shape_check(B, Nq, Nkv, Sq, Skv, D, scale);
+    if (sc != QBSA_OK) return sc;
+  }
+  if (Sq == 0) return QBSA_OK;
+  HostPathState* hp = nullptr;
+  qbsa_status st = host_path_state(&hp);
+  if (st != QBSA_OK) return st;
+
+  const int group = Nq / Nkv;
+  const int nqb = (Sq + 127) / 128, nkb = (Skv + 127) / 128;
+  const size_t sq = static_cast<size_t>(Sq), skv = static_cast<size_t>(Skv), dd = static_cast<size_t>(D);
+  // per-head sizes in bytes of every tensor; the device copies keep the host layout
+  const size_t q_h = sq * dd, k_h = skv * dd, qs_h = nqb * 4ull, ks_h = nkb * 4ull, vs_h = dd * 4,
+               m_h = static_cast<size_t>(nqb) * nkb, o_h = sq * dd * 2, st_h = sq * 4;
+  const size_t nq = static_cast<size_t>(B) * Nq, nk = static_cast<size_t>(B) * Nkv;
+  const size_t off_q = 0, off_k = off_q + round256(nq * q_h), off_v = off_k + round256(nk * k_h),
+               off_qs = off_v + round256(nk * k_h), off_ks = off_qs + round256(nq * qs_h),
+               off_vs = off_ks + round256(nk * ks_h), off_m = off_vs + round256(nk * vs_h),
+               off_o = off_m + round256(nq * m_h), off_mx = off_o + round256(nq * o_h),
+               off_sm = off_mx + round256(softmax_max ? nq * st_h : 0),
+               total = off_sm + round256(softmax_sum ? nq * st_h : 0);
+
+  cudaStream_t sc = static_cast<cudaStream_t>(stream);
+  cudaEvent_t ev_ready = nullptr, ev_in = nullptr, ev_comp = nullptr, ev_done = nullptr;
+  uint8_t* dbuf = nullptr;
+  cudaError_t e = cudaSuccess;
+  const char* what = nullptr;
+  auto ok = [&](cudaError_t r, const char* w) {
+    if (r != cudaSuccess && e == cudaSuccess) {
+      e = r;
+      what = w;
+    }
+    return e == cudaSuccess;
+  };
+  if (ok(cudaEventCreateWithFlags(&ev_ready, cudaEventDisableTiming), "cudaEventCreate") &&
+      ok(cudaEventCreateWithFlags(&ev_in, cudaEventDisableTiming), "cudaEventCreate") &&
+      ok(cudaEventCreateWithFlags(&ev_comp, cudaEventDisableTiming), "cudaEventCreate") &&
+      ok(cudaEventCreateWithFlags(&ev_done, cudaEventDisableTiming), "cudaEventCreate") &&
+      ok(cudaMallocFromPoolAsync(reinterpret_cast<void**>(&dbuf), total, hp->pool, sc), "cudaMallocFromPoolAsync") &&
+      ok(cudaEventRecord(ev_ready, sc), "cudaEventRecord") &&
+      ok(cudaStreamWaitEvent(hp->s_in, ev_ready, 0), "cudaStreamWaitEvent")) {
+    // chunks: whole GQA groups of kv heads [g0, g1) of one batch entry
+    const int per_b = std::max(1, std::min(Nkv, (n_chunks + B - 1) / B));
+    const auto h2d = [&](size_t off, const void* host, size_t bytes) {
+      return ok(cudaMemcpyAsync(dbuf + off, host, bytes, cudaMemcpyHostToDevice, hp->s_in), "cudaMemcpyAsync (in)");
+    };
+    const auto d2h = [&](void* host, size_t off, size_t bytes) {
+      return ok(cudaMemcpyAsync(host, dbuf + off, bytes, cudaMemcpyDeviceToHost, hp->s_out), "cudaMemcpyAsync (out)");
+    };
+    for (int b = 0; b < B && e == cudaSuccess && st == QBSA_OK; ++b) {
+      for (int c = 0; c < per_b && e == cudaSuccess && st == QBSA_OK; ++c) {
+        const int g0 = static_cast<int>((int64_t)c * Nkv / per_b), g1 = static_cast<int>((int64_t)(c + 1) * Nkv / per_b);
+        if (g1 <= g0) continue;
+        const size_t hq0 = static_cast<size_t>(b) * Nq + static_cast<size_t>(g0) * group;  // first query head
+        const size_t hk0 = static_cast<size_t>(b) * Nkv + g0;                               // first kv head
+        const size_t nhq = static_cast<size_t>(g1 - g0) * group, nhk = static_cast<size_t>(g1 - g0);
+        const uint8_t* hq = reinterpret_cast<const uint8_t*>(q_i8);
+        const uint8_t* hk = reinterpret_cast<const uint8_t*>(k_i8);
+        const uint8_t* hqs = reinterpret_cast<const uint8_t*>(q_block_scale);
+        const uint8_t* hks = reinterpret_cast<const uint8_t*>(k_block_scale);
+        const uint8_t* hvs = reinterpret_cast<const uint8_t*>(v_channel_scale);
+        if (!(h2d(off_q + hq0 * q_h, hq + hq0 * q_h, nhq * q_h) && h2d(off_k + hk0 * k_h, hk + hk0 * k_h, nhk * k_h) &&
+              h2d(off_v + hk0 * k_h, v_fp8 + hk0 * k_h, nhk * k_h) &&
+              h2d(off_qs + hq0 * qs_h, hqs + hq0 * qs_h, nhq * qs_h) &&
+              h2d(off_ks + hk0 * ks_h, hks + hk0 * ks_h, nhk * ks_h) &&
+              h2d(off_vs + hk0 * vs_h, hvs + hk0 * vs_h, nhk * vs_h) &&
+              h2d(off_m + hq0 * m_h, block_mask + hq0 * m_h, nhq * m_h) &&
+              ok(cudaEventRecord(ev_in, hp->s_in), "cudaEventRecord") &&
+              ok(cudaStreamWaitEvent(sc, ev_in, 0), "cudaStreamWaitEvent")))
+          break;
+        st = qbsa_fwd(reinterpret_cast<const int8_t*>(dbuf + off_q + hq0 * q_h),
+                      reinterpret_cast<const int8_t*>(dbuf + off_k + hk0 * k_h),
+                      reinterpret_cast<const float*>(dbuf + off_qs + hq0 * qs_h),
+                      reinterpret_cast<const float*>(dbuf + off_ks + hk0 * ks_h), dbuf + off_v + hk0 * k_h,
+                      reinterpret_cast<const float*>(dbuf + off_vs + hk0 * vs_h), dbuf + off_m + hq0 * m_h, 1,
+                      static_cast<int>(nhq), static_cast<int>(nhk), Sq, Skv, D, scale, dbuf + off_o + hq0 * o_h,
+                      softmax_max ? reinterpret_cast<float*>(dbuf + off_mx + hq0 * st_h) : nullptr,
+                      softmax_sum ? reinterpret_cast<float*>(dbuf + off_sm + hq0 * st_h) : nullptr, stream);
+        if (st != QBSA_OK) break;
+        if (!(ok(cudaEventRecord(ev_comp, sc), "cudaEventRecord") &&
+              ok(cudaStreamWaitEvent(hp->s_out, ev_comp, 0), "cudaStreamWaitEvent") &&
+              d2h(static_cast<uint8_t*>(attention_out) + hq0 * o_h, off_o + hq0 * o_h, nhq * o_h) &&
+              (!softmax_max ||
+               d2h(reinterpret_cast<uint8_t*>(softmax_max) + hq0 * st_h, off_mx + hq0 * st_h, nhq * st_h)) &&
+              (!softmax_sum ||
+               d2h(reinterpret_cast<uint8_t*>(softmax_sum) + hq0 * st_h, off_sm + hq0 * st_h, nhq * st_h))))
+          break;
+      }
+    }
+    // the buffers go back to the pool once the last copy out has read them
+    ok(cudaEventRecord(ev_done, hp->s_out), "cudaEventRecord");
+    ok(cudaStreamWaitEvent(sc, ev_done, 0), "cudaStreamWaitEvent");
+  }
+  if (dbuf) {
+    const cudaError_t r = cudaFreeAsync(dbuf, sc);
+    ok(r, "cudaFreeAsync");
+  }
+  ok(cudaStreamSynchronize(sc), "cudaStreamSynchronize");
+  for (cudaEvent_t ev : {ev_ready, ev_in, ev_comp, ev_done})
+    if (ev) cudaEventDestroy(ev);
+  if (st != QBSA_OK) return st;
+  if (e != cudaSuccess) return cuda_fail(e, what ? what : "qbsa_fwd_host");
   return QBSA_OK;
 }
 

@@ -33,7 +33,7 @@ def test_every_declared_symbol_is_exported():
     raw = ctypes.CDLL(qb.LIB_PATH)
     for n in names:
         assert hasattr(raw, n), n
-    assert qb.lib().qbsa_version() == 102  # 1.02: qbsa_block_topk_keep added
+    assert qb.lib().qbsa_version() == 103  # 1.03: qbsa_fwd_host added
 
 
 @pytest.mark.parametrize("nkb", [1, 2, 5, 7, 64, 255, 512, 1024, 2048])
@@ -121,6 +121,22 @@ def test_qbsa_fwd_rejects_before_launch():
     bad = list(args)
     bad[11] = 300 * 1024
     assert L.qbsa_fwd(*bad) == 2
+
+
+def test_qbsa_fwd_host_rejects_before_any_device_work():
+    """The host-buffer entry point validates like qbsa_fwd (plus n_chunks) before it touches
+    the device, so these calls return without a GPU."""
+    fake = ctypes.c_void_p(0x10000)
+    L = qb.lib()
+    args = [fake] * 7 + [1, 2, 1, 256, 256, 128, 0.1, fake, None, None, 8, None]
+    for idx, val, status in [(12, 64, 2), (0, None, 1), (14, None, 1), (8, 3, 1), (11, 300 * 1024, 2),
+                             (17, 0, 1), (17, -2, 1), (13, float("nan"), 1)]:
+        bad = list(args)
+        bad[idx] = val
+        if idx == 8:
+            bad[9] = 2          # Nq = 3 is not a multiple of Nkv = 2
+        st = L.qbsa_fwd_host(*bad)
+        assert st == status, (idx, val, qb.lib().qbsa_last_error().decode())
 
 
 def test_block_estimation_rejects_before_launch():
