@@ -14,7 +14,10 @@
 // walks the union of the two ranges, so every K/V tile is loaded once for the tiles that
 // need it, and the two tiles take turns on one TMEM score buffer.
 //
-// CTA = 11 warps, as attn_pair_kernel:
+// CTA = 12 warps, the roles of attn_pair_kernel plus an idle warp that completes the third
+// warpgroup: after set-up that warpgroup gives registers back (setmaxnreg, 168 -> 64 per
+// thread) and the two softmax warpgroups take them (168 -> 216), which removes the softmax
+// loop's spills (this kernel's per-row mask state needs more registers than the unmasked one):
 //   warps 0-3 / 4-7  softmax of tile 0 / tile 1 (row 32*(warp%4)+lane, lazy O rescale);
 //                    epilogue: O / l staged in the tile's Q buffer and written by TMA stores
 //                    (BNSD / BSND), or stored row by row (TND, whose tiles may end inside the
@@ -22,6 +25,7 @@
 //   warp 8           TMA producer: the Q tiles once, then the union's K and V tiles.
 //   warp 9           TMEM owner + QK issuer, for each tile whose range holds key tile j.
 //   warp 10          P·V issuer, each P·V queued behind the same tile's next QK.
+//   warp 11          no work after set-up.
 // TMEM columns: O0 [0,128) O1 [128,256) S [256,384) P0 [384,448) P1 [448,512).
 //
 // CTA order: query heads in groups whose K/V fit in about 48 MB of L2; inside a group the
@@ -118,7 +122,14 @@ __device__ __forceinline__ PairWork pair_work(const PairMaskedParams& p) {
   return w;
 }
 
-__global__ void __launch_bounds__(352, 1) attn_pair_masked_kernel(const __grid_constant__ PairMaskedParams p) {
+struct PairMaskedCfg {
+  static constexpr int kThreads = 384;
+  static constexpr int kRegSoftmax = 216, kRegHelper = 64;  // per thread, after set-up
+};
+static_assert(2 * 128 * PairMaskedCfg::kRegSoftmax + 128 * PairMaskedCfg::kRegHelper <= PairMaskedCfg::kThreads * 168,
+              "register shares above what a 168-register launch holds");
+
+__global__ void __launch_bounds__(384, 1) attn_pair_masked_kernel(const __grid_constant__ PairMaskedParams p) {
   using C = PairCfg;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
@@ -184,6 +195,8 @@ __global__ void __launch_bounds__(352, 1) attn_pair_masked_kernel(const __grid_c
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  if (warp >= 8) {
+  regs_dec<PairMaskedCfg::kRegHelper>();
   if (warp == C::kWarpProducer) {
     // ---------------------------------------------------------------- producer
     if (lane == 0 && nj > 0) {
@@ -320,7 +333,9 @@ __global__ void __launch_bounds__(352, 1) attn_pair_masked_kernel(const __grid_c
       mma_commit(bar(C::kBarDrain + 1));
       mbar_wait_drain(bar(C::kBarDrain + 1), 0);
     }
-  } else if (warp < 8) {
+  }
+  } else {
+    regs_inc<PairMaskedCfg::kRegSoftmax>();
     // ---------------------------------------------------------------- softmax warps
     const int t = warp >> 2;
     const int quarter = warp & 3;

@@ -153,6 +153,21 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// Register reallocation between warpgroups (setmaxnreg): every warp of a warpgroup must run
+// the same instruction; an increase waits until the CTA's pool, which holds what the launch
+// gave (threads x registers per thread), has the registers, so the shares must add up to at
+// most that total.
+template <int N>
+__device__ __forceinline__ void regs_dec() {
+  static_assert(N % 8 == 0 && N >= 24 && N <= 256, "setmaxnreg count");
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_inc() {
+  static_assert(N % 8 == 0 && N >= 24 && N <= 256, "setmaxnreg count");
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ---------------------------------------------------------------------------------
 // tcgen05: TMEM allocation, MMA, commit, fences
 // ---------------------------------------------------------------------------------

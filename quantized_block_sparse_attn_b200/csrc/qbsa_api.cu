@@ -374,7 +374,7 @@ static qbsa_status attn_fwd_impl(const void* q, const void* k, const void* v, in
     const int64_t n_pw = n_pairs * Nq;
     if (n_pw == 0) return QBSA_OK;
     if ((st = set_smem(qbsa::attn_pair_masked_kernel, qbsa::PairCfg::kSmemBytes)) != QBSA_OK) return st;
-    qbsa::attn_pair_masked_kernel<<<dim3(static_cast<unsigned>(n_pw)), qbsa::PairCfg::kThreads,
+    qbsa::attn_pair_masked_kernel<<<dim3(static_cast<unsigned>(n_pw)), qbsa::PairMaskedCfg::kThreads,
                                     qbsa::PairCfg::kSmemBytes, s>>>(pp);
     return check_launch("attn_pair_masked_kernel launch");
   }
