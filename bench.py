@@ -6,8 +6,8 @@ B=1, N=40, S=65536, D=128, INT8 Q/K per 128-token block, E4M3 V per channel, 128
 block mask keeping 10% of the blocks per (head, query block) with the diagonal kept.
 Reported beside it under "extra": bf16 block-sparse attention on the same mask, the
 on-GPU quantisers, block-mask estimation, dense bf16 attention at S=61440 (the video
-workload) and S=65536, the causal (B=2, N=16, S=4096) and GQA varlen TND workloads,
-and the sweep over S = 8K..128K at keep 0.1 and 0.5 plus dense at each S (the metric's
+workload) and S=65536, the causal (B=2, N=16, S=4096) and GQA varlen TND workloads, an
+explicit atten_mask and a pse (B=1, N=16, S=4096), and the sweep over S = 8K..128K at keep 0.1 and 0.5 plus dense at each S (the metric's
 "vs S" curve; ``--no-sweep`` skips it).  Lines whose inputs fit in L2 flush it (a
 256 MB write) before every timed step and time each step alone.
 
@@ -458,6 +458,7 @@ def run_ours(args):
         extra["dense_S65536"] = dense_line(device, stream, 65536, 2, 10, bf16_peak, dist)
         extra["causal"] = causal_line(device, stream, bf16_peak, flush)
         extra["gqa_varlen"] = gqa_varlen_line(device, stream, bf16_peak, flush)
+        extra["explicit_mask"] = explicit_mask_line(device, stream, bf16_peak, hbm_peak, flush)
     # ---------------------------------------------------------------- the metric's curve over S
     if not args.no_sweep:
         sweep = []
@@ -650,6 +651,40 @@ def gqa_varlen_line(device, stream, bf16_peak, flush):
             "executed_tflops": executed / ms / 1e9, "useful_tflops": useful / ms / 1e9,
             "pct_of_bf16_peak": 100 * executed / ms / 1e9 / bf16_peak, "kernel": "attn_pair_masked_kernel",
             "l2": "flushed before each step"}
+
+
+def explicit_mask_line(device, stream, bf16_peak, hbm_peak, flush):
+    """attn_fwd with an explicit atten_mask (SS, shared by all heads) or a pse (BNSS), B=1,
+    N=16, S=4096, D=128, BNSD, sparse_mode 0, with stats: the one-tile kernel's general path."""
+    import torch
+    import quantized_block_sparse_attn_b200 as qb
+    from workloads import device_iid_normal_bf16, random_atten_mask
+    B, N, S, D, seed = 1, 16, 4096, 128, 41
+    q, k, v = (device_iid_normal_bf16(seed, t, (B, N, S, D), device) for t in range(3))
+    mask = torch.from_numpy(random_atten_mask(seed, (S, S), 0.5)).to(device)
+    pse = device_iid_normal_bf16(seed, 3, (B, N, S, S), device)
+    out = torch.empty_like(q)
+    smax = torch.empty((B, N, S), dtype=torch.float32, device=device)
+    ssum = torch.empty_like(smax)
+    flops = 4.0 * D * S * S * B * N
+    res = {}
+    for name, kw, extra_bytes in (("atten_mask_SS", dict(atten_mask=mask, mask_shape="SS"), S * S),
+                                  ("pse_BNSS", dict(pse=pse), 2 * B * N * S * S)):
+        def step(kw=kw):
+            qb.attn_fwd(q, k, v, N, "BNSD", scale=D ** -0.5, out=out, softmax_max=smax, softmax_sum=ssum, **kw)
+
+        total, per, _ = time_steps(step, 20, 3, stream, flush=flush)
+        qb.check(device)
+        ms = total / 20
+        res[name] = {"ms": ms, "tflops": flops / ms / 1e9, "pct_of_bf16_peak": 100 * flops / ms / 1e9 / bf16_peak,
+                     "extra_input_bytes": extra_bytes,
+                     "extra_input_frac_of_hbm": extra_bytes / (ms * 1e-3) / 1e9 / hbm_peak}
+    del q, k, v, mask, pse, out, smax, ssum
+    torch.cuda.empty_cache()
+    res.update({"workload": f"attn_fwd bf16 B={B} N={N} S={S} D={D} BNSD, sparse_mode 0, stats; an SS atten_mask "
+                            "(half the keys masked, iid) or a BNSS pse (iid N(0,1))",
+                "kernel": "attn_dense_kernel<128, general>", "l2": "flushed before each step"})
+    return res
 
 
 def quantize_line(device, stream, S, hbm_peak):

@@ -9,18 +9,20 @@
 // attn_pair_kernel (two query tiles per CTA, attn_pair.cuh); this kernel serves every
 // other case, including bsa_fwd's block lists.
 //
-// CTA = 10 warps:
-//   warp 0      TMA producer: Q once, then K/V tiles into a 2-stage ring each.
-//   warp 1      TMEM owner + MMA issuer (one thread): S = Q Kᵀ (kind::f16, SS) into a
-//               double-buffered f32 TMEM tile, then O += P V (kind::f16, A = P from
-//               TMEM, B = V from shared memory, MN-major).
-//   warps 2..9  softmax: query row 32*(warp%4)+lane (the warp's TMEM lane quarter);
-//               warps 2..5 own score columns [0,64), warps 6..9 columns [64,128) of
+// CTA = 12 warps (three warpgroups).  After set-up the third warpgroup gives registers back
+// (setmaxnreg, 168 -> 64 per thread) and the two softmax warpgroups take them (168 -> 216):
+//   warps 0..7  softmax: query row 32*(warp%4)+lane (the warp's TMEM lane quarter);
+//               warps 0..3 own score columns [0,64), warps 4..7 columns [64,128) of
 //               the same rows, and exchange their partial row maxima through shared
 //               memory (a 64-thread named barrier per lane quarter).  O is rescaled in
 //               TMEM only when the running max grew by more than 2^8 (the lagging
 //               reference cancels in O / l; the statistics are corrected at the end).
 //               P goes to TMEM as bf16; the epilogue normalises O and stores it.
+//   warp 8      TMA producer: Q once, then K/V tiles into a 2-stage ring each.
+//   warp 9      MMA issuer (one thread): S = Q Kᵀ (kind::f16, SS) into a
+//               double-buffered f32 TMEM tile, then O += P V (kind::f16, A = P from
+//               TMEM, B = V from shared memory, MN-major).
+//   warps 10-11 no work after set-up (warp 1 allocates and frees TMEM around the roles).
 // TMEM columns: S0 [0,128) S1 [128,256) O [256,256+D) P0 [384,448) P1 [448,512).
 //
 // CTA order: query heads are taken in groups whose K/V fit in about 48 MB of L2; in
@@ -61,6 +63,8 @@ struct DenseParams {
   // optional 128x128 block mask [B, Nq, n_qtiles, mask_nkb] (1 = compute), BNSD / BSND only
   const uint8_t* block_mask;
   int mask_nkb;
+  int mask_v16;  // atten_mask rows and base 16-byte aligned (S_kv % 16 == 0): vector reads
+  int pse_v16;   // pse rows and base 16-byte aligned (S_kv % 8 == 0): vector reads
   float scale;
   // TND tables (sequences in processing order)
   int n_seq;
@@ -102,9 +106,12 @@ struct DenseCfg {
   // TMEM columns
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256, kColP0 = 384, kColP1 = 448;
-  static constexpr int kThreads = 320;
+  static constexpr int kThreads = 384;
   static constexpr int kSoftmaxThreads = 256;
 };
+constexpr int kDenseRegSoftmax = 216, kDenseRegHelper = 64;  // per thread, after set-up
+static_assert(2 * 128 * kDenseRegSoftmax + 128 * kDenseRegHelper <= 384 * 168,
+              "register shares above what a 168-register launch holds");
 
 struct DenseWork {
   int b, h, qt;
@@ -154,8 +161,15 @@ __device__ __forceinline__ DenseWork dense_work(const DenseParams& p) {
   return w;
 }
 
-template <int D>
-__global__ void __launch_bounds__(320, 1) attn_dense_kernel(const __grid_constant__ DenseParams p) {
+// Word k (0..3, a compile-time index after unrolling) of a 16-byte vector.
+__device__ __forceinline__ uint32_t u4_word(const uint4& v, int k) {
+  return k == 0 ? v.x : k == 1 ? v.y : k == 2 ? v.z : v.w;
+}
+
+// kGeneral: an explicit atten_mask or pse is present (the instantiation without them carries
+// none of their code, which the other callers would otherwise pay for in the softmax loop).
+template <int D, bool kGeneral>
+__global__ void __launch_bounds__(384, 1) attn_dense_kernel(const __grid_constant__ DenseParams p) {
   using C = DenseCfg<D>;
   constexpr int kHalfD = D / 2;  // O columns per softmax half
   extern __shared__ uint8_t smem_raw[];
@@ -175,7 +189,7 @@ __global__ void __launch_bounds__(320, 1) attn_dense_kernel(const __grid_constan
   const int g = w.h / p.group;
   const Band band = band_of(p.sparse_mode, p.pre_tokens, p.next_tokens, w.sq, w.skv);
   const TileRange tr = tile_range(w.qt, w.sq, w.skv, band);
-  const bool general_mask = (p.atten_mask != nullptr) || (p.pse != nullptr);
+  constexpr bool general_mask = kGeneral;
   uint16_t* klist = reinterpret_cast<uint16_t*>(smem + C::kListOff);
   int* count_slot = reinterpret_cast<int*>(smem + C::kMiscOff + 8);
 
@@ -225,7 +239,9 @@ __global__ void __launch_bounds__(320, 1) attn_dense_kernel(const __grid_constan
   const int n = listed ? *count_slot : tr.kt_end - tr.kt_begin;
   auto ktile = [&](int it) -> int { return listed ? static_cast<int>(klist[it]) : tr.kt_begin + it; };
 
-  if (warp == 0) {
+  if (warp >= 8) {
+  regs_dec<kDenseRegHelper>();
+  if (warp == 8) {
     // ---------------------------------------------------------------- producer
     if (lane == 0 && n > 0) {
       const uint64_t pol_q = l2_policy_evict_first();
@@ -251,7 +267,7 @@ __global__ void __launch_bounds__(320, 1) attn_dense_kernel(const __grid_constan
                       sub * 64, kv_row, g, w.coord_b, pol_kv);
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == 9) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0 && n > 0) {
       constexpr uint32_t idesc_qk = idesc_bf16(128, 128, false);
@@ -297,14 +313,16 @@ __global__ void __launch_bounds__(320, 1) attn_dense_kernel(const __grid_constan
       }
       if (ok && issue_pv(n - 1)) mma_commit(bar(C::kBarOFinal));
     }
+  }
   } else {
+    regs_inc<kDenseRegSoftmax>();
     // ---------------------------------------------------------------- softmax warps
     const int quarter = warp & 3;
-    const int half = (warp - 2) >> 2;  // 0: score columns [0,64), 1: [64,128)
+    const int half = warp >> 2;  // 0: score columns [0,64), 1: [64,128)
     const int row = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const int64_t i_loc = (int64_t)w.qt * kTile + row;  // query index inside the sequence
-    const bool has_pse = p.pse != nullptr;
+    const bool has_pse = kGeneral && p.pse != nullptr;
     const float vs = has_pse ? 1.0f : p.scale;  // score = value * vs
     const float c = vs * 1.4426950408889634f;   // value -> log2 domain
     const float kNegInf = -__int_as_float(0x7f800000);
@@ -314,10 +332,31 @@ __global__ void __launch_bounds__(320, 1) attn_dense_kernel(const __grid_constan
 
     const uint8_t* mrow = nullptr;
     const __nv_bfloat16* prow = nullptr;
-    if (p.atten_mask && i_loc < w.sq)
+    if (kGeneral && p.atten_mask && i_loc < w.sq)
       mrow = p.atten_mask + w.b * p.m_batch_stride + w.h * p.m_head_stride + i_loc * p.m_row_stride;
     if (has_pse && i_loc < w.sq)
       prow = p.pse + w.b * p.p_batch_stride + w.h * p.p_head_stride + i_loc * p.p_row_stride;
+
+    // atten_mask / pse of a key tile: this row's 64 mask bytes / 64 pse values of the half,
+    // read with 16-byte loads one tile ahead (issued once the previous tile's values are
+    // used) when the rows are aligned and the half lies inside S_kv; otherwise, and for a
+    // ragged last tile, element by element when the tile is processed
+    uint4 mpre[4], ppre[8];
+    const bool mrow_v = mrow != nullptr && p.mask_v16;
+    const bool prow_v = prow != nullptr && p.pse_v16;
+    auto fetch = [&](int it2) {
+      const int64_t c0 = (int64_t)ktile(it2) * kTile + half * 64;
+      if (c0 + 64 > w.skv) return;
+      if (mrow_v) {
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) mpre[q4] = __ldg(reinterpret_cast<const uint4*>(mrow + c0) + q4);
+      }
+      if (prow_v) {
+#pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4) ppre[q4] = __ldg(reinterpret_cast<const uint4*>(prow + c0) + q4);
+      }
+    };
+    if (kGeneral && n > 0 && (mrow_v || prow_v)) fetch(0);
 
     float m_ref = kNegInf, m_true = kNegInf, l = 0.f;  // l: this half's partial sum
     bool ok = true;
@@ -342,20 +381,40 @@ __global__ void __launch_bounds__(320, 1) attn_dense_kernel(const __grid_constan
       if (!full || general_mask) {
         const int64_t col0 = (int64_t)kt * kTile + half * 64;
         const int64_t clo = j_lo - col0, chi = j_hi - col0;
+        const bool inside = col0 + 64 <= w.skv;  // then the prefetched vectors hold this tile
+        if (kGeneral && has_pse) {
+          if (prow_v && inside) {
 #pragma unroll
-        for (int x = 0; x < 64; ++x) {
-          float v = sv[x];
-          if (has_pse) {
-            const int64_t j = col0 + x;
-            v = v * p.scale + ((prow && j < w.skv) ? __bfloat162float(prow[j]) : 0.f);
+            for (int x = 0; x < 64; ++x) {
+              const uint32_t wd = u4_word(ppre[x >> 3], (x >> 1) & 3);
+              sv[x] = sv[x] * p.scale + __uint_as_float((x & 1) ? (wd & 0xffff0000u) : (wd << 16));
+            }
+          } else {
+#pragma unroll
+            for (int x = 0; x < 64; ++x) {
+              const int64_t j = col0 + x;
+              sv[x] = sv[x] * p.scale + ((prow && j < w.skv) ? __bfloat162float(prow[j]) : 0.f);
+            }
           }
-          bool keep = (x >= clo) && (x <= chi);
-          if (mrow) {
-            const int64_t j = col0 + x;
-            keep = keep && (j < w.skv) && (mrow[j] == 0);
-          }
-          sv[x] = keep ? v : kNegInf;
         }
+        if (kGeneral && mrow_v && inside) {
+#pragma unroll
+          for (int x = 0; x < 64; ++x) {
+            const uint32_t byte = (u4_word(mpre[x >> 4], (x >> 2) & 3) >> (8 * (x & 3))) & 0xffu;
+            sv[x] = (x >= clo && x <= chi && byte == 0u) ? sv[x] : kNegInf;
+          }
+        } else {
+#pragma unroll
+          for (int x = 0; x < 64; ++x) {
+            bool keep = (x >= clo) && (x <= chi);
+            if (kGeneral && mrow) {
+              const int64_t j = col0 + x;
+              keep = keep && (j < w.skv) && (mrow[j] == 0);
+            }
+            sv[x] = keep ? sv[x] : kNegInf;
+          }
+        }
+        if (kGeneral && (mrow_v || prow_v) && it + 1 < n) fetch(it + 1);
       }
       const float pmax = max64(sv);
       // combine the two halves of the row

@@ -113,13 +113,20 @@ struct SeqInfo {
   int q_start, q_len, kv_start, kv_len;
 };
 
+template <int D, bool kGeneral>
+qbsa_status launch_dense_as(qbsa::DenseParams& prm, int64_t n_work, cudaStream_t stream) {
+  using C = qbsa::DenseCfg<D>;
+  qbsa_status st = set_smem(qbsa::attn_dense_kernel<D, kGeneral>, C::kSmemBytes);
+  if (st != QBSA_OK) return st;
+  qbsa::attn_dense_kernel<D, kGeneral>
+      <<<dim3(static_cast<unsigned>(n_work)), C::kThreads, C::kSmemBytes, stream>>>(prm);
+  return check_launch("attn_dense_kernel launch");
+}
+
 template <int D>
 qbsa_status launch_dense(qbsa::DenseParams& prm, int64_t n_work, cudaStream_t stream) {
-  using C = qbsa::DenseCfg<D>;
-  qbsa_status st = set_smem(qbsa::attn_dense_kernel<D>, C::kSmemBytes);
-  if (st != QBSA_OK) return st;
-  qbsa::attn_dense_kernel<D><<<dim3(static_cast<unsigned>(n_work)), C::kThreads, C::kSmemBytes, stream>>>(prm);
-  return check_launch("attn_dense_kernel launch");
+  const bool general = prm.atten_mask != nullptr || prm.pse != nullptr;
+  return general ? launch_dense_as<D, true>(prm, n_work, stream) : launch_dense_as<D, false>(prm, n_work, stream);
 }
 
 }  // namespace
@@ -248,12 +255,14 @@ static qbsa_status attn_fwd_impl(const void* q, const void* k, const void* v, in
     prm.m_batch_stride = (mask_shape == QBSA_MASK_SS) ? 0
                          : (mask_shape == QBSA_MASK_B1SS) ? (int64_t)Sq * Skv
                                                           : (int64_t)Nq * Sq * Skv;
+    prm.mask_v16 = (Skv % 16 == 0) && (reinterpret_cast<uintptr_t>(atten_mask) % 16 == 0);
   }
   if (pse) {
     prm.pse = static_cast<const __nv_bfloat16*>(pse);
     prm.p_row_stride = Skv;
     prm.p_head_stride = (int64_t)Sq * Skv;
     prm.p_batch_stride = pse_batch_bcast ? 0 : (int64_t)Nq * Sq * Skv;
+    prm.pse_v16 = (Skv % 8 == 0) && (reinterpret_cast<uintptr_t>(pse) % 16 == 0);
   }
 
   int64_t n_rank = 0;

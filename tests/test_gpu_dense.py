@@ -91,6 +91,29 @@ def test_dense_pse(bcast):
     _run_and_compare(q, k, v, "BNSD", Nq, D ** -0.5, 3, pse=pse)
 
 
+@pytest.mark.parametrize("shape", ["SS", "B1SS", "BNSS"])
+@pytest.mark.parametrize("D", [64, 128])
+def test_dense_atten_mask_aligned_rows(shape, D):
+    """S_kv % 16 == 0: the mask rows are read as 16-byte vectors a key tile ahead, except the
+    half-tiles that run past S_kv (384..399 here), which are read byte by byte."""
+    B, Nq, Sq, Skv = 2, 2, 300, 400
+    q, k, v = _bnsd(18, B, Nq, Nq, Sq, Skv, D)
+    mshape = {"SS": (Sq, Skv), "B1SS": (B, 1, Sq, Skv), "BNSS": (B, Nq, Sq, Skv)}[shape]
+    mask = random_atten_mask(18, mshape, 0.4)
+    _run_and_compare(q, k, v, "BNSD", Nq, D ** -0.5, 0, 200, 150, mask=mask, mask_shape=shape)
+
+
+@pytest.mark.parametrize("Skv", [400, 403])
+def test_dense_pse_and_mask_together(Skv):
+    """pse and atten_mask in one call, with vector reads of both (S_kv = 400) or of neither
+    (S_kv = 403: rows not 16-byte aligned)."""
+    B, Nq, Sq, D = 1, 2, 260, 128
+    q, k, v = _bnsd(19, B, Nq, Nq, Sq, Skv, D)
+    pse = random_pse_bf16(19, (B, Nq, Sq, Skv), 2.0)
+    mask = random_atten_mask(19, (Sq, Skv), 0.3)
+    _run_and_compare(q, k, v, "BNSD", Nq, D ** -0.5, 0, mask=mask, mask_shape="SS", pse=pse)
+
+
 @pytest.mark.parametrize("D", [64, 128])
 def test_dense_tnd_gqa_causal(D):
     lens_q, lens_k = [100, 300, 77, 256], [130, 300, 50, 256]
