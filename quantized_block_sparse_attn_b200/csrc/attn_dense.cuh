@@ -63,8 +63,13 @@ struct DenseParams {
   // optional 128x128 block mask [B, Nq, n_qtiles, mask_nkb] (1 = compute), BNSD / BSND only
   const uint8_t* block_mask;
   int mask_nkb;
-  int mask_v16;  // atten_mask rows and base 16-byte aligned (S_kv % 16 == 0): vector reads
-  int pse_v16;   // pse rows and base 16-byte aligned (S_kv % 8 == 0): vector reads
+  // atten_mask / pse tiles by TMA (rows 16-byte aligned: S_kv % 16 == 0 for the mask, % 8 for
+  // pse, bases 16-byte aligned); otherwise the softmax warps read them element by element
+  int mask_tma, pse_tma;
+  int mask_heads, mask_batches;  // the mask's head / batch coordinates apply (B1SS, BNSS)
+  int pse_batches;               // pse's batch coordinate applies (no batch broadcast)
+  CUtensorMap tm_m;  // uint8 {S_kv, S_q, heads, batches}, box {128, 128, 1, 1}, SW128
+  CUtensorMap tm_p;  // bf16 {S_kv, S_q, N_q, batches}, box {64, 128, 1, 1}, SW128
   float scale;
   // TND tables (sequences in processing order)
   int n_seq;
@@ -83,7 +88,9 @@ struct DenseCfg {
   static constexpr int kQOff = 0;
   static constexpr int kKOff = kQOff + kTileBytes;
   static constexpr int kVOff = kKOff + kStages * kTileBytes;
-  static constexpr int kXOff = kVOff + kStages * kTileBytes;  // row-max exchange: float [2][2][128]
+  static constexpr int kMOff = kVOff + kStages * kTileBytes;  // atten_mask tile, 128 x 128 bytes
+  static constexpr int kPOff = kMOff + kTile * 128;             // pse tile, two 128 x 64 bf16 halves
+  static constexpr int kXOff = kPOff + kTile * 256;             // row-max exchange: float [2][2][128]
   static constexpr int kListOff = kXOff + 2 * 2 * 128 * 4;    // uint16 kept K tiles (block mask)
   static constexpr int kMaxListed = 2048;
   static constexpr int kBarOff = kListOff + kMaxListed * 2;
@@ -98,7 +105,9 @@ struct DenseCfg {
   static constexpr int kBarPFull = kBarSFree + 2;         // 2
   static constexpr int kBarPVDone = kBarPFull + 2;        // 1
   static constexpr int kBarOFinal = kBarPVDone + 1;       // 1: last P·V done (single use)
-  static constexpr int kNumBars = kBarOFinal + 1;
+  static constexpr int kBarMFull = kBarOFinal + 1;        // 1: atten_mask / pse tile landed
+  static constexpr int kBarMEmpty = kBarMFull + 1;        // 1: ... and read by every softmax thread
+  static constexpr int kNumBars = kBarMEmpty + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   // + alignment slack; at least 120 KB so that one CTA holds an SM (and its 512 TMEM columns)
   static constexpr int kSmemUsed = kMiscOff + 16 + 1024;
@@ -109,6 +118,9 @@ struct DenseCfg {
   static constexpr int kThreads = 384;
   static constexpr int kSoftmaxThreads = 256;
 };
+static_assert(DenseCfg<128>::kSmemBytes <= 232448, "shared memory above the 227 KB opt-in limit");
+static_assert(DenseCfg<128>::kMOff % 1024 == 0 && DenseCfg<64>::kMOff % 1024 == 0,
+              "swizzled buffers must start on 1024-byte boundaries");
 constexpr int kDenseRegSoftmax = 216, kDenseRegHelper = 64;  // per thread, after set-up
 static_assert(2 * 128 * kDenseRegSoftmax + 128 * kDenseRegHelper <= 384 * 168,
               "register shares above what a 168-register launch holds");
@@ -222,10 +234,14 @@ __global__ void __launch_bounds__(384, 1) attn_dense_kernel(const __grid_constan
     }
     mbar_init(bar(C::kBarPVDone), 1);
     mbar_init(bar(C::kBarOFinal), 1);
+    mbar_init(bar(C::kBarMFull), 1);
+    mbar_init(bar(C::kBarMEmpty), C::kSoftmaxThreads);
     fence_mbar_init();
     tma_prefetch_desc(&p.tm_q);
     tma_prefetch_desc(&p.tm_k);
     tma_prefetch_desc(&p.tm_v);
+    if (kGeneral && p.mask_tma) tma_prefetch_desc(&p.tm_m);
+    if (kGeneral && p.pse_tma) tma_prefetch_desc(&p.tm_p);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
@@ -247,6 +263,7 @@ __global__ void __launch_bounds__(384, 1) attn_dense_kernel(const __grid_constan
       const uint64_t pol_q = l2_policy_evict_first();
       const uint64_t pol_kv = l2_policy_evict_last();
       const int q_row = static_cast<int>(w.q_row0 + (int64_t)w.qt * kTile);
+      int n_staged = 0;  // atten_mask / pse tiles loaded
       mbar_arrive_expect_tx(bar(C::kBarQFull), C::kTileBytes);
       for (int sub = 0; sub < D / 64; ++sub)
         tma_load_4d(base + C::kQOff + sub * C::kSubBytes, &p.tm_q, bar(C::kBarQFull), sub * 64, q_row, w.h,
@@ -265,7 +282,26 @@ __global__ void __launch_bounds__(384, 1) attn_dense_kernel(const __grid_constan
         for (int sub = 0; sub < D / 64; ++sub)
           tma_load_4d(base + C::kVOff + s * C::kTileBytes + sub * C::kSubBytes, &p.tm_v, bar(C::kBarVFull + s),
                       sub * 64, kv_row, g, w.coord_b, pol_kv);
+        if (kGeneral && (p.mask_tma || p.pse_tma)) {
+          // atten_mask / pse tile of (query tile, key tile) into the single-stage buffer, once
+          // every softmax thread has read the previous one (early in its step, so the load has
+          // about a step to land)
+          if (it >= 1 && !mbar_wait(bar(C::kBarMEmpty), (it - 1) & 1, abort_flag)) break;
+          const int kc = ktile(it) * kTile, qr = w.qt * kTile;
+          mbar_arrive_expect_tx(bar(C::kBarMFull), (p.mask_tma ? kTile * 128 : 0) + (p.pse_tma ? kTile * 256 : 0));
+          if (p.mask_tma)  // shared by heads (and batches) for SS / B1SS: keep it in L2
+            tma_load_4d(base + C::kMOff, &p.tm_m, bar(C::kBarMFull), kc, qr, p.mask_heads ? w.h : 0,
+                        p.mask_batches ? w.b : 0, pol_kv);
+          if (p.pse_tma) {
+            for (int hf = 0; hf < 2; ++hf)
+              tma_load_4d(base + C::kPOff + hf * kTile * 128, &p.tm_p, bar(C::kBarMFull), kc + 64 * hf, qr, w.h,
+                          p.pse_batches ? w.b : 0, pol_q);
+          }
+          n_staged = it + 1;
+        }
       }
+      // the last staged tile has landed before the CTA can exit (matters only after an abort)
+      if (n_staged > 0) mbar_wait_drain(bar(C::kBarMFull), static_cast<uint32_t>(n_staged - 1) & 1);
     }
   } else if (warp == 9) {
     // ---------------------------------------------------------------- MMA issuer
@@ -337,26 +373,14 @@ __global__ void __launch_bounds__(384, 1) attn_dense_kernel(const __grid_constan
     if (has_pse && i_loc < w.sq)
       prow = p.pse + w.b * p.p_batch_stride + w.h * p.p_head_stride + i_loc * p.p_row_stride;
 
-    // atten_mask / pse of a key tile: this row's 64 mask bytes / 64 pse values of the half,
-    // read with 16-byte loads one tile ahead (issued once the previous tile's values are
-    // used) when the rows are aligned and the half lies inside S_kv; otherwise, and for a
-    // ragged last tile, element by element when the tile is processed
-    uint4 mpre[4], ppre[8];
-    const bool mrow_v = mrow != nullptr && p.mask_v16;
-    const bool prow_v = prow != nullptr && p.pse_v16;
-    auto fetch = [&](int it2) {
-      const int64_t c0 = (int64_t)ktile(it2) * kTile + half * 64;
-      if (c0 + 64 > w.skv) return;
-      if (mrow_v) {
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) mpre[q4] = __ldg(reinterpret_cast<const uint4*>(mrow + c0) + q4);
-      }
-      if (prow_v) {
-#pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4) ppre[q4] = __ldg(reinterpret_cast<const uint4*>(prow + c0) + q4);
-      }
-    };
-    if (kGeneral && n > 0 && (mrow_v || prow_v)) fetch(0);
+    // atten_mask / pse of a key tile: staged by the producer (TMA, 128-byte swizzle: 16-byte
+    // chunk c of row r sits at chunk c ^ (r % 8)), this row's 64 mask bytes / 64 pse values of
+    // the half read as four / eight 16-byte loads; without TMA (unaligned rows) read element by
+    // element from global memory
+    const bool m_tma = kGeneral && p.mask_tma, p_tma = kGeneral && p.pse_tma;
+    const uint32_t m_line = base + C::kMOff + row * 128;
+    const uint32_t p_line = base + C::kPOff + half * (kTile * 128) + row * 128;
+    const uint32_t swz = static_cast<uint32_t>(row & 7);
 
     float m_ref = kNegInf, m_true = kNegInf, l = 0.f;  // l: this half's partial sum
     bool ok = true;
@@ -381,13 +405,20 @@ __global__ void __launch_bounds__(384, 1) attn_dense_kernel(const __grid_constan
       if (!full || general_mask) {
         const int64_t col0 = (int64_t)kt * kTile + half * 64;
         const int64_t clo = j_lo - col0, chi = j_hi - col0;
-        const bool inside = col0 + 64 <= w.skv;  // then the prefetched vectors hold this tile
+        if (kGeneral && (m_tma || p_tma)) {
+          if (ok) ok = mbar_wait(bar(C::kBarMFull), static_cast<uint32_t>(it) & 1, abort_flag);
+        }
         if (kGeneral && has_pse) {
-          if (prow_v && inside) {
+          if (p_tma) {
 #pragma unroll
-            for (int x = 0; x < 64; ++x) {
-              const uint32_t wd = u4_word(ppre[x >> 3], (x >> 1) & 3);
-              sv[x] = sv[x] * p.scale + __uint_as_float((x & 1) ? (wd & 0xffff0000u) : (wd << 16));
+            for (int c8 = 0; c8 < 8; ++c8) {
+              const uint4 v8 = lds128(p_line + ((static_cast<uint32_t>(c8) ^ swz) << 4));
+#pragma unroll
+              for (int y = 0; y < 8; ++y) {
+                const int x = 8 * c8 + y;
+                const uint32_t wd = u4_word(v8, y >> 1);
+                sv[x] = sv[x] * p.scale + __uint_as_float((y & 1) ? (wd & 0xffff0000u) : (wd << 16));
+              }
             }
           } else {
 #pragma unroll
@@ -397,11 +428,30 @@ __global__ void __launch_bounds__(384, 1) attn_dense_kernel(const __grid_constan
             }
           }
         }
-        if (kGeneral && mrow_v && inside) {
+        uint32_t nz[16];  // bit 8k+7 of nz[i]: mask byte 4i+k of this half is nonzero (masked)
+        if (m_tma) {
 #pragma unroll
-          for (int x = 0; x < 64; ++x) {
-            const uint32_t byte = (u4_word(mpre[x >> 4], (x >> 2) & 3) >> (8 * (x & 3))) & 0xffu;
-            sv[x] = (x >= clo && x <= chi && byte == 0u) ? sv[x] : kNegInf;
+          for (int c4 = 0; c4 < 4; ++c4) {
+            const uint4 v4 = lds128(m_line + ((static_cast<uint32_t>(4 * half + c4) ^ swz) << 4));
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const uint32_t wd = u4_word(v4, k);
+              nz[4 * c4 + k] = (((wd & 0x7f7f7f7fu) + 0x7f7f7f7fu) | wd) & 0x80808080u;
+            }
+          }
+        }
+        if (kGeneral && (m_tma || p_tma)) mbar_arrive(bar(C::kBarMEmpty));  // this thread is done with the tile
+        if (m_tma) {
+          if (clo <= 0 && chi >= 63) {  // the whole half lies inside this row's band
+#pragma unroll
+            for (int x = 0; x < 64; ++x)
+              sv[x] = ((nz[x >> 2] >> (8 * (x & 3) + 7)) & 1u) ? kNegInf : sv[x];
+          } else {
+#pragma unroll
+            for (int x = 0; x < 64; ++x) {
+              const bool keep = (x >= clo) && (x <= chi) && !((nz[x >> 2] >> (8 * (x & 3) + 7)) & 1u);
+              sv[x] = keep ? sv[x] : kNegInf;
+            }
           }
         } else {
 #pragma unroll
@@ -414,7 +464,6 @@ __global__ void __launch_bounds__(384, 1) attn_dense_kernel(const __grid_constan
             sv[x] = keep ? sv[x] : kNegInf;
           }
         }
-        if (kGeneral && (mrow_v || prow_v) && it + 1 < n) fetch(it + 1);
       }
       const float pmax = max64(sv);
       // combine the two halves of the row

@@ -128,6 +128,13 @@ __device__ __forceinline__ uint64_t l2_policy_evict_first() {
 }
 
 // 4-D tiled load into this CTA's shared memory, completing on an mbarrier.
+// 16-byte shared-memory load.
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
 __device__ __forceinline__ void tma_load_4d(uint32_t dst, const void* map, uint32_t bar, int c0, int c1,
                                             int c2, int c3, uint64_t policy) {
   asm volatile(

@@ -255,14 +255,12 @@ static qbsa_status attn_fwd_impl(const void* q, const void* k, const void* v, in
     prm.m_batch_stride = (mask_shape == QBSA_MASK_SS) ? 0
                          : (mask_shape == QBSA_MASK_B1SS) ? (int64_t)Sq * Skv
                                                           : (int64_t)Nq * Sq * Skv;
-    prm.mask_v16 = (Skv % 16 == 0) && (reinterpret_cast<uintptr_t>(atten_mask) % 16 == 0);
   }
   if (pse) {
     prm.pse = static_cast<const __nv_bfloat16*>(pse);
     prm.p_row_stride = Skv;
     prm.p_head_stride = (int64_t)Sq * Skv;
     prm.p_batch_stride = pse_batch_bcast ? 0 : (int64_t)Nq * Sq * Skv;
-    prm.pse_v16 = (Skv % 8 == 0) && (reinterpret_cast<uintptr_t>(pse) % 16 == 0);
   }
 
   int64_t n_rank = 0;
@@ -298,6 +296,24 @@ static qbsa_status attn_fwd_impl(const void* q, const void* k, const void* v, in
   if ((st = make_map(&prm.tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, qd, qs, 64)) != QBSA_OK) return st;
   if ((st = make_map(&prm.tm_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, k, kd, ks, 64)) != QBSA_OK) return st;
   if ((st = make_map(&prm.tm_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, v, kd, ks, 64)) != QBSA_OK) return st;
+  // atten_mask / pse tiles by TMA when their rows and bases are 16-byte aligned
+  if (atten_mask && Skv % 16 == 0 && reinterpret_cast<uintptr_t>(atten_mask) % 16 == 0) {
+    prm.mask_heads = mask_shape == QBSA_MASK_BNSS;
+    prm.mask_batches = mask_shape != QBSA_MASK_SS;
+    const uint64_t nh = prm.mask_heads ? Nq : 1, nb = prm.mask_batches ? B : 1;
+    const uint64_t md[4] = {(uint64_t)Skv, (uint64_t)Sq, nh, nb};
+    const uint64_t ms[3] = {(uint64_t)Skv, (uint64_t)Sq * Skv, nh * Sq * Skv};
+    if ((st = make_map(&prm.tm_m, CU_TENSOR_MAP_DATA_TYPE_UINT8, atten_mask, md, ms, 128)) != QBSA_OK) return st;
+    prm.mask_tma = 1;
+  }
+  if (pse && Skv % 8 == 0 && reinterpret_cast<uintptr_t>(pse) % 16 == 0) {
+    prm.pse_batches = !pse_batch_bcast;
+    const uint64_t nb = prm.pse_batches ? B : 1;
+    const uint64_t pd[4] = {(uint64_t)Skv, (uint64_t)Sq, (uint64_t)Nq, nb};
+    const uint64_t ps[3] = {2ull * Skv, 2ull * Sq * Skv, 2ull * Nq * Sq * Skv};
+    if ((st = make_map(&prm.tm_p, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, pse, pd, ps, 64)) != QBSA_OK) return st;
+    prm.pse_tma = 1;
+  }
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // unmasked D = 128 BNSD / BSND (no atten_mask, pse or block mask; a band that covers

@@ -247,6 +247,18 @@ def test_dense_lazy_rescale_growing_k(B, Nq, Nkv, Sq, Skv, D, mode, layout):
     _run_and_compare(q, k, v, layout, Nq, D ** -0.5, mode)
 
 
+@pytest.mark.parametrize("D", [64, 128])
+def test_dense_lazy_rescale_growing_k_mask_and_pse(D):
+    """The one-tile kernel's atten_mask / pse instantiation through the same rescales: S_kv =
+    688 (a multiple of 16, so all but the last half-tile are read as vectors)."""
+    B, Nq, Nkv, Sq, Skv = 1, 2, 1, 300, 688
+    q, k, v = _bnsd(15, B, Nq, Nkv, Sq, Skv, D)
+    k, v = _growing_k(k, Skv), _quarter(v)
+    mask = random_atten_mask(15, (B, 1, Sq, Skv), 0.2)
+    pse = random_pse_bf16(15, (B, Nq, Sq, Skv), 0.5)
+    _run_and_compare(q, k, v, "BNSD", Nq, D ** -0.5, 0, mask=mask, mask_shape="B1SS", pse=pse)
+
+
 def test_bsa_lazy_rescale_growing_k():
     """bsa_fwd (one-tile kernel walking a kept-block list) with the row max growing past the
     rescale threshold at several kept K tiles."""
