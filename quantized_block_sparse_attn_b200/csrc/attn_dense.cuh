@@ -453,16 +453,16 @@ __global__ void __launch_bounds__(384, 1) attn_dense_kernel(const __grid_constan
               sv[x] = keep ? sv[x] : kNegInf;
             }
           }
-        } else {
+        } else if (kGeneral && mrow) {
 #pragma unroll
           for (int x = 0; x < 64; ++x) {
-            bool keep = (x >= clo) && (x <= chi);
-            if (kGeneral && mrow) {
-              const int64_t j = col0 + x;
-              keep = keep && (j < w.skv) && (mrow[j] == 0);
-            }
+            const int64_t j = col0 + x;
+            const bool keep = (x >= clo) && (x <= chi) && (j < w.skv) && (mrow[j] == 0);
             sv[x] = keep ? sv[x] : kNegInf;
           }
+        } else if (!(clo <= 0 && chi >= 63)) {  // band only, and the half is not inside it
+#pragma unroll
+          for (int x = 0; x < 64; ++x) sv[x] = (x >= clo && x <= chi) ? sv[x] : kNegInf;
         }
       }
       const float pmax = max64(sv);
