@@ -186,11 +186,11 @@ qbsa_status qbsa_quantize_qk(const void* x_bf16, int B, int N, int S, int D, int
  * scales fp32 [B, N, D].  D in {64, 128, 256} (else QBSA_ERR_UNSUPPORTED); v, codes and
  * scales 16-byte aligned.
  * Two streaming passes: the column maxima of every (head, chunk), folded per head, then
- * the codes (heads in reverse order, so the first chunks read are still in L2).  They need
- * B*N*D * 4 bytes of scratch for the per-head maxima, which this call takes from the
- * stream-ordered allocator (cudaMallocAsync / cudaFreeAsync on `stream`, the device's
- * current memory pool) and zeroes; an allocation failure returns QBSA_ERR_CUDA before the
- * kernels are queued.
+ * the codes.  They need B*N*D * 4 bytes of scratch for the per-head maxima, which this call
+ * takes, stream-ordered on `stream`, from a memory pool the library keeps per device
+ * (created on first use; it keeps its memory between calls, so after the first call of a
+ * size no allocation maps memory) and zeroes; an allocation failure returns QBSA_ERR_CUDA
+ * before the kernels are queued.
  */
 qbsa_status qbsa_quantize_v(const void* v_bf16, int B, int N, int S, int D, uint8_t* codes, float* scales,
                             void* stream);

@@ -581,6 +581,40 @@ qbsa_status v_quant_launch(const qbsa::VQuantParams& prm, int D, cudaStream_t st
   return check_launch("v_quant_kernel launch");
 }
 
+// Per device, a stream-ordered memory pool whose memory stays with the library between calls
+// (release threshold: everything), so that scratch and staging buffers cost no fresh
+// allocation after the first call of a size.  (The device's default pool returns its memory
+// at every synchronisation, after which each allocation maps memory again on the host's
+// issue path.)
+constexpr int kPoolDevices = 64;
+std::mutex g_pool_mu;
+cudaMemPool_t g_pool[kPoolDevices] = {};
+
+qbsa_status library_pool(cudaMemPool_t* out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kPoolDevices) return fail(QBSA_ERR_UNSUPPORTED, "device ordinal %d", dev);
+  std::lock_guard<std::mutex> lock(g_pool_mu);
+  if (!g_pool[dev]) {
+    cudaMemPoolProps props;
+    memset(&props, 0, sizeof(props));
+    props.allocType = cudaMemAllocationTypePinned;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t pool = nullptr;
+    if ((e = cudaMemPoolCreate(&pool, &props)) != cudaSuccess) return cuda_fail(e, "cudaMemPoolCreate");
+    uint64_t keep = ~0ull;
+    if ((e = cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep)) != cudaSuccess) {
+      cudaMemPoolDestroy(pool);
+      return cuda_fail(e, "cudaMemPoolSetAttribute");
+    }
+    g_pool[dev] = pool;
+  }
+  *out = g_pool[dev];
+  return QBSA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -592,9 +626,11 @@ qbsa_status qbsa_quantize_v(const void* v_bf16, int B, int N, int S, int D, uint
   if (st != QBSA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const size_t bytes = static_cast<size_t>(v_quant_scratch_words(prm.H, D)) * sizeof(unsigned int);
+  cudaMemPool_t pool = nullptr;
+  if ((st = library_pool(&pool)) != QBSA_OK) return st;
   void* scratch = nullptr;
-  cudaError_t e = cudaMallocAsync(&scratch, bytes, s);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaMallocAsync (V quantiser scratch)");
+  cudaError_t e = cudaMallocFromPoolAsync(&scratch, bytes, pool, s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMallocFromPoolAsync (V quantiser scratch)");
   e = cudaMemsetAsync(scratch, 0, bytes, s);
   if (e != cudaSuccess) {
     cudaFreeAsync(scratch, s);
@@ -805,8 +841,8 @@ qbsa_status qbsa_check(void* stream) {
 // ------------------------------------------------------------------------------
 //
 // Per device the library keeps two non-blocking copy streams (host -> device, device ->
-// host) and a stream-ordered memory pool whose memory is kept between calls, so that a
-// call's device buffers cost no fresh allocation after the first call of that size.
+// host); the call's device buffers come from the library's memory pool (above), so they cost
+// no fresh allocation after the first call of that size.
 
 namespace {
 
@@ -833,15 +869,8 @@ qbsa_status host_path_state(HostPathState** out) {
       return cuda_fail(e, "cudaStreamCreateWithFlags (copy-in stream)");
     if ((e = cudaStreamCreateWithFlags(&st.s_out, cudaStreamNonBlocking)) != cudaSuccess)
       return cuda_fail(e, "cudaStreamCreateWithFlags (copy-out stream)");
-    cudaMemPoolProps props;
-    memset(&props, 0, sizeof(props));
-    props.allocType = cudaMemAllocationTypePinned;
-    props.location.type = cudaMemLocationTypeDevice;
-    props.location.id = dev;
-    if ((e = cudaMemPoolCreate(&st.pool, &props)) != cudaSuccess) return cuda_fail(e, "cudaMemPoolCreate");
-    uint64_t keep = ~0ull;
-    if ((e = cudaMemPoolSetAttribute(st.pool, cudaMemPoolAttrReleaseThreshold, &keep)) != cudaSuccess)
-      return cuda_fail(e, "cudaMemPoolSetAttribute");
+    const qbsa_status ps = library_pool(&st.pool);
+    if (ps != QBSA_OK) return ps;
     st.ready = true;
   }
   *out = &st;
