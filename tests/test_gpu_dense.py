@@ -103,10 +103,11 @@ def test_dense_atten_mask_aligned_rows(shape, D):
     _run_and_compare(q, k, v, "BNSD", Nq, D ** -0.5, 0, 200, 150, mask=mask, mask_shape=shape)
 
 
-@pytest.mark.parametrize("Skv", [400, 403])
+@pytest.mark.parametrize("Skv", [400, 403, 408])
 def test_dense_pse_and_mask_together(Skv):
-    """pse and atten_mask in one call, with vector reads of both (S_kv = 400) or of neither
-    (S_kv = 403: rows not 16-byte aligned)."""
+    """pse and atten_mask in one call: both staged by TMA (S_kv = 400), neither (S_kv = 403:
+    rows not 16-byte aligned, read element by element), or only pse (S_kv = 408: pse rows
+    16-byte aligned, mask rows not)."""
     B, Nq, Sq, D = 1, 2, 260, 128
     q, k, v = _bnsd(19, B, Nq, Nq, Sq, Skv, D)
     pse = random_pse_bf16(19, (B, Nq, Sq, Skv), 2.0)
