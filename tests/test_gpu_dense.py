@@ -103,6 +103,18 @@ def test_dense_atten_mask_aligned_rows(shape, D):
     _run_and_compare(q, k, v, "BNSD", Nq, D ** -0.5, 0, 200, 150, mask=mask, mask_shape=shape)
 
 
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("Skv", [16, 96])
+def test_dense_mask_and_pse_short_keys(Skv, D):
+    """S_kv below one key tile but 16-byte aligned: the staged mask / pse boxes extend past the
+    rows (the copy fills the rest, which the S_kv bound masks)."""
+    B, Nq, Sq = 2, 2, 130
+    q, k, v = _bnsd(20, B, Nq, Nq, Sq, Skv, D)
+    pse = random_pse_bf16(20, (1, Nq, Sq, Skv), 1.0)
+    mask = random_atten_mask(20, (B, Nq, Sq, Skv), 0.3)
+    _run_and_compare(q, k, v, "BNSD", Nq, D ** -0.5, 0, mask=mask, mask_shape="BNSS", pse=pse)
+
+
 @pytest.mark.parametrize("Skv", [400, 403, 408])
 def test_dense_pse_and_mask_together(Skv):
     """pse and atten_mask in one call: both staged by TMA (S_kv = 400), neither (S_kv = 403:
