@@ -75,3 +75,20 @@ def test_reference_arm_prints_the_contract_line():
 
 def bench_metric():
     return _bench().METRIC
+
+
+def test_visited_tiles_count_matches_the_oracle_tile_sets():
+    """The executed-FLOP count of the causal and TND lines counts the key tiles the schedule
+    visits; it must equal the number of (query tile, key tile) pairs holding a kept element,
+    counted by brute force over the element mask."""
+    from oracle import dense
+    from quantized_block_sparse_attn_b200 import build
+    build.build()
+    bench = _bench()
+    for sq, skv, mode in [(4096, 4096, 3), (1024, 1024, 3), (5000, 5000, 3), (300, 333, 2), (333, 300, 3),
+                          (640, 640, 0)]:
+        want = sum(len(vis) for vis, _ in dense.tile_sets(sq, skv, mode))
+        assert bench._visited_tiles(sq, skv, mode) == want, (sq, skv, mode)
+    # causal, equal lengths: tile t visits t + 1 key tiles
+    n = 4096 // 128
+    assert bench._visited_tiles(4096, 4096, 3) == n * (n + 1) // 2
