@@ -256,100 +256,100 @@ __global__ void __launch_bounds__(384, 1) attn_dense_kernel(const __grid_constan
   auto ktile = [&](int it) -> int { return listed ? static_cast<int>(klist[it]) : tr.kt_begin + it; };
 
   if (warp >= 8) {
-  regs_dec<kDenseRegHelper>();
-  if (warp == 8) {
-    // ---------------------------------------------------------------- producer
-    if (lane == 0 && n > 0) {
-      const uint64_t pol_q = l2_policy_evict_first();
-      const uint64_t pol_kv = l2_policy_evict_last();
-      const int q_row = static_cast<int>(w.q_row0 + (int64_t)w.qt * kTile);
-      int n_staged = 0;  // atten_mask / pse tiles loaded
-      mbar_arrive_expect_tx(bar(C::kBarQFull), C::kTileBytes);
-      for (int sub = 0; sub < D / 64; ++sub)
-        tma_load_4d(base + C::kQOff + sub * C::kSubBytes, &p.tm_q, bar(C::kBarQFull), sub * 64, q_row, w.h,
-                    w.coord_b, pol_q);
-      for (int it = 0; it < n; ++it) {
-        const int s = it % C::kStages;
-        const uint32_t ph = (it / C::kStages) & 1;
-        const int kv_row = static_cast<int>(w.kv_row0 + (int64_t)ktile(it) * kTile);
-        if (it >= C::kStages && !mbar_wait(bar(C::kBarKEmpty + s), ph ^ 1, abort_flag)) break;
-        mbar_arrive_expect_tx(bar(C::kBarKFull + s), C::kTileBytes);
+    regs_dec<kDenseRegHelper>();
+    if (warp == 8) {
+      // ---------------------------------------------------------------- producer
+      if (lane == 0 && n > 0) {
+        const uint64_t pol_q = l2_policy_evict_first();
+        const uint64_t pol_kv = l2_policy_evict_last();
+        const int q_row = static_cast<int>(w.q_row0 + (int64_t)w.qt * kTile);
+        int n_staged = 0;  // atten_mask / pse tiles loaded
+        mbar_arrive_expect_tx(bar(C::kBarQFull), C::kTileBytes);
         for (int sub = 0; sub < D / 64; ++sub)
-          tma_load_4d(base + C::kKOff + s * C::kTileBytes + sub * C::kSubBytes, &p.tm_k, bar(C::kBarKFull + s),
-                      sub * 64, kv_row, g, w.coord_b, pol_kv);
-        if (it >= C::kStages && !mbar_wait(bar(C::kBarVEmpty + s), ph ^ 1, abort_flag)) break;
-        mbar_arrive_expect_tx(bar(C::kBarVFull + s), C::kTileBytes);
-        for (int sub = 0; sub < D / 64; ++sub)
-          tma_load_4d(base + C::kVOff + s * C::kTileBytes + sub * C::kSubBytes, &p.tm_v, bar(C::kBarVFull + s),
-                      sub * 64, kv_row, g, w.coord_b, pol_kv);
-        if (kGeneral && (p.mask_tma || p.pse_tma)) {
-          // atten_mask / pse tile of (query tile, key tile) into the single-stage buffer, once
-          // every softmax thread has read the previous one (early in its step, so the load has
-          // about a step to land)
-          if (it >= 1 && !mbar_wait(bar(C::kBarMEmpty), (it - 1) & 1, abort_flag)) break;
-          const int kc = ktile(it) * kTile, qr = w.qt * kTile;
-          mbar_arrive_expect_tx(bar(C::kBarMFull), (p.mask_tma ? kTile * 128 : 0) + (p.pse_tma ? kTile * 256 : 0));
-          if (p.mask_tma)  // shared by heads (and batches) for SS / B1SS: keep it in L2
-            tma_load_4d(base + C::kMOff, &p.tm_m, bar(C::kBarMFull), kc, qr, p.mask_heads ? w.h : 0,
-                        p.mask_batches ? w.b : 0, pol_kv);
-          if (p.pse_tma) {
-            for (int hf = 0; hf < 2; ++hf)
-              tma_load_4d(base + C::kPOff + hf * kTile * 128, &p.tm_p, bar(C::kBarMFull), kc + 64 * hf, qr, w.h,
-                          p.pse_batches ? w.b : 0, pol_q);
+          tma_load_4d(base + C::kQOff + sub * C::kSubBytes, &p.tm_q, bar(C::kBarQFull), sub * 64, q_row, w.h,
+                      w.coord_b, pol_q);
+        for (int it = 0; it < n; ++it) {
+          const int s = it % C::kStages;
+          const uint32_t ph = (it / C::kStages) & 1;
+          const int kv_row = static_cast<int>(w.kv_row0 + (int64_t)ktile(it) * kTile);
+          if (it >= C::kStages && !mbar_wait(bar(C::kBarKEmpty + s), ph ^ 1, abort_flag)) break;
+          mbar_arrive_expect_tx(bar(C::kBarKFull + s), C::kTileBytes);
+          for (int sub = 0; sub < D / 64; ++sub)
+            tma_load_4d(base + C::kKOff + s * C::kTileBytes + sub * C::kSubBytes, &p.tm_k, bar(C::kBarKFull + s),
+                        sub * 64, kv_row, g, w.coord_b, pol_kv);
+          if (it >= C::kStages && !mbar_wait(bar(C::kBarVEmpty + s), ph ^ 1, abort_flag)) break;
+          mbar_arrive_expect_tx(bar(C::kBarVFull + s), C::kTileBytes);
+          for (int sub = 0; sub < D / 64; ++sub)
+            tma_load_4d(base + C::kVOff + s * C::kTileBytes + sub * C::kSubBytes, &p.tm_v, bar(C::kBarVFull + s),
+                        sub * 64, kv_row, g, w.coord_b, pol_kv);
+          if (kGeneral && (p.mask_tma || p.pse_tma)) {
+            // atten_mask / pse tile of (query tile, key tile) into the single-stage buffer, once
+            // every softmax thread has read the previous one (early in its step, so the load has
+            // about a step to land)
+            if (it >= 1 && !mbar_wait(bar(C::kBarMEmpty), (it - 1) & 1, abort_flag)) break;
+            const int kc = ktile(it) * kTile, qr = w.qt * kTile;
+            mbar_arrive_expect_tx(bar(C::kBarMFull), (p.mask_tma ? kTile * 128 : 0) + (p.pse_tma ? kTile * 256 : 0));
+            if (p.mask_tma)  // shared by heads (and batches) for SS / B1SS: keep it in L2
+              tma_load_4d(base + C::kMOff, &p.tm_m, bar(C::kBarMFull), kc, qr, p.mask_heads ? w.h : 0,
+                          p.mask_batches ? w.b : 0, pol_kv);
+            if (p.pse_tma) {
+              for (int hf = 0; hf < 2; ++hf)
+                tma_load_4d(base + C::kPOff + hf * kTile * 128, &p.tm_p, bar(C::kBarMFull), kc + 64 * hf, qr, w.h,
+                            p.pse_batches ? w.b : 0, pol_q);
+            }
+            n_staged = it + 1;
           }
-          n_staged = it + 1;
         }
+        // the last staged tile has landed before the CTA can exit (matters only after an abort)
+        if (n_staged > 0) mbar_wait_drain(bar(C::kBarMFull), static_cast<uint32_t>(n_staged - 1) & 1);
       }
-      // the last staged tile has landed before the CTA can exit (matters only after an abort)
-      if (n_staged > 0) mbar_wait_drain(bar(C::kBarMFull), static_cast<uint32_t>(n_staged - 1) & 1);
-    }
-  } else if (warp == 9) {
-    // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0 && n > 0) {
-      constexpr uint32_t idesc_qk = idesc_bf16(128, 128, false);
-      constexpr uint32_t idesc_pv = idesc_bf16(128, D, true);
-      bool ok = mbar_wait(bar(C::kBarQFull), 0, abort_flag);
-      auto issue_pv = [&](int j) -> bool {
-        const int bj = j & 1;
-        const int s = j % C::kStages;
-        if (!mbar_wait(bar(C::kBarPFull + bj), (j >> 1) & 1, abort_flag)) return false;
-        if (!mbar_wait(bar(C::kBarVFull + s), (j / C::kStages) & 1, abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t vbase = base + C::kVOff + s * C::kTileBytes;
-        const uint32_t pcol = bj ? C::kColP1 : C::kColP0;
-#pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk) {
-          // B = V tile, MN-major: 16 key rows per step (2048 B), D-halves 16 KB apart
-          const uint64_t bdesc = sdesc_sw128(vbase + kk * 2048, C::kSubBytes, 1024);
-          mma_f16_ts(tmem + C::kColO, tmem + pcol + kk * 8, bdesc, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+    } else if (warp == 9) {
+      // ---------------------------------------------------------------- MMA issuer
+      if (lane == 0 && n > 0) {
+        constexpr uint32_t idesc_qk = idesc_bf16(128, 128, false);
+        constexpr uint32_t idesc_pv = idesc_bf16(128, D, true);
+        bool ok = mbar_wait(bar(C::kBarQFull), 0, abort_flag);
+        auto issue_pv = [&](int j) -> bool {
+          const int bj = j & 1;
+          const int s = j % C::kStages;
+          if (!mbar_wait(bar(C::kBarPFull + bj), (j >> 1) & 1, abort_flag)) return false;
+          if (!mbar_wait(bar(C::kBarVFull + s), (j / C::kStages) & 1, abort_flag)) return false;
+          tc_fence_after();
+          const uint32_t vbase = base + C::kVOff + s * C::kTileBytes;
+          const uint32_t pcol = bj ? C::kColP1 : C::kColP0;
+  #pragma unroll
+          for (int kk = 0; kk < kTile / 16; ++kk) {
+            // B = V tile, MN-major: 16 key rows per step (2048 B), D-halves 16 KB apart
+            const uint64_t bdesc = sdesc_sw128(vbase + kk * 2048, C::kSubBytes, 1024);
+            mma_f16_ts(tmem + C::kColO, tmem + pcol + kk * 8, bdesc, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(bar(C::kBarPVDone));
+          mma_commit(bar(C::kBarVEmpty + s));
+          return true;
+        };
+        const uint32_t qbase = base + C::kQOff;
+        for (int it = 0; ok && it < n; ++it) {
+          const int s = it % C::kStages;
+          const int bi = it & 1;
+          if (!mbar_wait(bar(C::kBarKFull + s), (it / C::kStages) & 1, abort_flag)) { ok = false; break; }
+          if (it >= 2 && !mbar_wait(bar(C::kBarSFree + bi), ((it - 2) >> 1) & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t kbase = base + C::kKOff + s * C::kTileBytes;
+          const uint32_t scol = bi ? C::kColS1 : C::kColS0;
+  #pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            // A = Q, B = K, both K-major: 16 elements (32 B) per step inside a 64-wide column
+            const uint32_t off = (kk >> 2) * C::kSubBytes + (kk & 3) * 32;
+            mma_f16_ss(tmem + scol, sdesc_sw128(qbase + off, 16, 1024), sdesc_sw128(kbase + off, 16, 1024), idesc_qk,
+                       kk > 0 ? 1u : 0u);
+          }
+          mma_commit(bar(C::kBarSFull + bi));
+          mma_commit(bar(C::kBarKEmpty + s));
+          if (it >= 1 && !issue_pv(it - 1)) { ok = false; break; }
         }
-        mma_commit(bar(C::kBarPVDone));
-        mma_commit(bar(C::kBarVEmpty + s));
-        return true;
-      };
-      const uint32_t qbase = base + C::kQOff;
-      for (int it = 0; ok && it < n; ++it) {
-        const int s = it % C::kStages;
-        const int bi = it & 1;
-        if (!mbar_wait(bar(C::kBarKFull + s), (it / C::kStages) & 1, abort_flag)) { ok = false; break; }
-        if (it >= 2 && !mbar_wait(bar(C::kBarSFree + bi), ((it - 2) >> 1) & 1, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t kbase = base + C::kKOff + s * C::kTileBytes;
-        const uint32_t scol = bi ? C::kColS1 : C::kColS0;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          // A = Q, B = K, both K-major: 16 elements (32 B) per step inside a 64-wide column
-          const uint32_t off = (kk >> 2) * C::kSubBytes + (kk & 3) * 32;
-          mma_f16_ss(tmem + scol, sdesc_sw128(qbase + off, 16, 1024), sdesc_sw128(kbase + off, 16, 1024), idesc_qk,
-                     kk > 0 ? 1u : 0u);
-        }
-        mma_commit(bar(C::kBarSFull + bi));
-        mma_commit(bar(C::kBarKEmpty + s));
-        if (it >= 1 && !issue_pv(it - 1)) { ok = false; break; }
+        if (ok && issue_pv(n - 1)) mma_commit(bar(C::kBarOFinal));
       }
-      if (ok && issue_pv(n - 1)) mma_commit(bar(C::kBarOFinal));
     }
-  }
   } else {
     regs_inc<kDenseRegSoftmax>();
     // ---------------------------------------------------------------- softmax warps

@@ -196,144 +196,145 @@ __global__ void __launch_bounds__(384, 1) attn_pair_masked_kernel(const __grid_c
   const uint32_t tmem = *tmem_slot;
 
   if (warp >= 8) {
-  regs_dec<PairMaskedCfg::kRegHelper>();
-  if (warp == C::kWarpProducer) {
-    // ---------------------------------------------------------------- producer
-    if (lane == 0 && nj > 0) {
-      const uint64_t pol_q = l2_policy_evict_first();
-      const uint64_t pol_kv = l2_policy_evict_last();
-      mbar_arrive_expect_tx(bar(C::kBarQFull), C::kTileBytes * ((n0 > 0) + (n1 > 0)));
-      for (int t = 0; t < 2; ++t) {
-        if ((t ? n1 : n0) == 0) continue;
-        const int qrow = static_cast<int>(w.q_row0 + (int64_t)(2 * w.pr + t) * kTile);
-        for (int sub = 0; sub < 2; ++sub)
-          tma_load_4d(base + C::kQOff + t * C::kTileBytes + sub * C::kSubBytes, &p.tm_q, bar(C::kBarQFull),
-                      sub * 64, qrow, h, w.coord_b, pol_q);
-      }
-      int kq = 0, vq = 0;  // K / V copies issued
-      for (int jj = 0; jj < nj; ++jj) {
-        const int kv_row = static_cast<int>(w.kv_row0 + (int64_t)(ub + jj) * kTile);
-        const int sk = jj % C::kKStages, sv = jj % C::kVStages;
-        if (jj >= C::kKStages &&
-            !mbar_wait(bar(C::kBarKEmpty + sk), (static_cast<uint32_t>(jj / C::kKStages) & 1) ^ 1, abort_flag))
-          break;
-        mbar_arrive_expect_tx(bar(C::kBarKFull + sk), C::kTileBytes);
-        for (int sub = 0; sub < 2; ++sub)
-          tma_load_4d(base + C::kKOff + sk * C::kTileBytes + sub * C::kSubBytes, &p.tm_k, bar(C::kBarKFull + sk),
-                      sub * 64, kv_row, g, w.coord_b, pol_kv);
-        ++kq;
-        if (jj >= C::kVStages &&
-            !mbar_wait(bar(C::kBarVEmpty + sv), (static_cast<uint32_t>(jj / C::kVStages) & 1) ^ 1, abort_flag))
-          break;
-        mbar_arrive_expect_tx(bar(C::kBarVFull + sv), C::kTileBytes);
-        for (int sub = 0; sub < 2; ++sub)
-          tma_load_4d(base + C::kVOff + sv * C::kTileBytes + sub * C::kSubBytes, &p.tm_v, bar(C::kBarVFull + sv),
-                      sub * 64, kv_row, g, w.coord_b, pol_kv);
-        ++vq;
-      }
-      // let the copies still in flight land before the CTA can exit (matters only after an
-      // abort): an older copy's stage was reused, so it had been consumed
-      for (int q = max(0, kq - C::kKStages); q < kq; ++q)
-        mbar_wait_drain(bar(C::kBarKFull + q % C::kKStages), static_cast<uint32_t>(q / C::kKStages) & 1);
-      for (int q = max(0, vq - C::kVStages); q < vq; ++q)
-        mbar_wait_drain(bar(C::kBarVFull + q % C::kVStages), static_cast<uint32_t>(q / C::kVStages) & 1);
-      mbar_wait_drain(bar(C::kBarQFull), 0);
-    }
-  } else if (warp == C::kWarpQK) {
-    // ---------------------------------------------------------------- QK issuer
-    if (lane == 0 && nj > 0) {
-      constexpr uint32_t idesc_qk = idesc_bf16(128, 128, false);
-      bool ok = mbar_wait(bar(C::kBarQFull), 0, abort_flag);
-      int prev_t = -1, prev_l = 0;  // reader of the S buffer's current contents (tile, local block)
-      for (int jj = 0; ok && jj < nj; ++jj) {
-        const int j = ub + jj;
-        const int s = jj % C::kKStages;
-        if (!mbar_wait(bar(C::kBarKFull + s), static_cast<uint32_t>(jj / C::kKStages) & 1, abort_flag)) {
-          ok = false;
-          break;
-        }
-        const uint32_t kbase = base + C::kKOff + s * C::kTileBytes;
-#pragma unroll
+    regs_dec<PairMaskedCfg::kRegHelper>();
+    if (warp == C::kWarpProducer) {
+      // ---------------------------------------------------------------- producer
+      if (lane == 0 && nj > 0) {
+        const uint64_t pol_q = l2_policy_evict_first();
+        const uint64_t pol_kv = l2_policy_evict_last();
+        mbar_arrive_expect_tx(bar(C::kBarQFull), C::kTileBytes * ((n0 > 0) + (n1 > 0)));
         for (int t = 0; t < 2; ++t) {
-          const int kb = t ? kb1 : kb0, ke = t ? ke1 : ke0;
-          if (!ok || j < kb || j >= ke) continue;
-          const int lt = j - kb;
-          if (prev_t >= 0 && !mbar_wait(bar(C::kBarSFree + prev_t), static_cast<uint32_t>(prev_l) & 1, abort_flag)) {
+          if ((t ? n1 : n0) == 0) continue;
+          const int qrow = static_cast<int>(w.q_row0 + (int64_t)(2 * w.pr + t) * kTile);
+          for (int sub = 0; sub < 2; ++sub)
+            tma_load_4d(base + C::kQOff + t * C::kTileBytes + sub * C::kSubBytes, &p.tm_q, bar(C::kBarQFull),
+                        sub * 64, qrow, h, w.coord_b, pol_q);
+        }
+        int kq = 0, vq = 0;  // K / V copies issued
+        for (int jj = 0; jj < nj; ++jj) {
+          const int kv_row = static_cast<int>(w.kv_row0 + (int64_t)(ub + jj) * kTile);
+          const int sk = jj % C::kKStages, sv = jj % C::kVStages;
+          if (jj >= C::kKStages &&
+              !mbar_wait(bar(C::kBarKEmpty + sk), (static_cast<uint32_t>(jj / C::kKStages) & 1) ^ 1, abort_flag))
+            break;
+          mbar_arrive_expect_tx(bar(C::kBarKFull + sk), C::kTileBytes);
+          for (int sub = 0; sub < 2; ++sub)
+            tma_load_4d(base + C::kKOff + sk * C::kTileBytes + sub * C::kSubBytes, &p.tm_k, bar(C::kBarKFull + sk),
+                        sub * 64, kv_row, g, w.coord_b, pol_kv);
+          ++kq;
+          if (jj >= C::kVStages &&
+              !mbar_wait(bar(C::kBarVEmpty + sv), (static_cast<uint32_t>(jj / C::kVStages) & 1) ^ 1, abort_flag))
+            break;
+          mbar_arrive_expect_tx(bar(C::kBarVFull + sv), C::kTileBytes);
+          for (int sub = 0; sub < 2; ++sub)
+            tma_load_4d(base + C::kVOff + sv * C::kTileBytes + sub * C::kSubBytes, &p.tm_v, bar(C::kBarVFull + sv),
+                        sub * 64, kv_row, g, w.coord_b, pol_kv);
+          ++vq;
+        }
+        // let the copies still in flight land before the CTA can exit (matters only after an
+        // abort): an older copy's stage was reused, so it had been consumed
+        for (int q = max(0, kq - C::kKStages); q < kq; ++q)
+          mbar_wait_drain(bar(C::kBarKFull + q % C::kKStages), static_cast<uint32_t>(q / C::kKStages) & 1);
+        for (int q = max(0, vq - C::kVStages); q < vq; ++q)
+          mbar_wait_drain(bar(C::kBarVFull + q % C::kVStages), static_cast<uint32_t>(q / C::kVStages) & 1);
+        mbar_wait_drain(bar(C::kBarQFull), 0);
+      }
+    } else if (warp == C::kWarpQK) {
+      // ---------------------------------------------------------------- QK issuer
+      if (lane == 0 && nj > 0) {
+        constexpr uint32_t idesc_qk = idesc_bf16(128, 128, false);
+        bool ok = mbar_wait(bar(C::kBarQFull), 0, abort_flag);
+        int prev_t = -1, prev_l = 0;  // reader of the S buffer's current contents (tile, local block)
+        for (int jj = 0; ok && jj < nj; ++jj) {
+          const int j = ub + jj;
+          const int s = jj % C::kKStages;
+          if (!mbar_wait(bar(C::kBarKFull + s), static_cast<uint32_t>(jj / C::kKStages) & 1, abort_flag)) {
             ok = false;
             break;
           }
-          tc_fence_after();
-          const uint32_t qbase = base + C::kQOff + t * C::kTileBytes;
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            // 16 elements (32 bytes) per step inside a 64-wide swizzle column
-            const uint32_t o = (kk >> 2) * C::kSubBytes + (kk & 3) * 32;
-            mma_f16_ss(tmem + C::kColS, sdesc_sw128(qbase + o, 16, 1024), sdesc_sw128(kbase + o, 16, 1024), idesc_qk,
-                       kk > 0 ? 1u : 0u);
+          const uint32_t kbase = base + C::kKOff + s * C::kTileBytes;
+  #pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            const int kb = t ? kb1 : kb0, ke = t ? ke1 : ke0;
+            if (!ok || j < kb || j >= ke) continue;
+            const int lt = j - kb;
+            if (prev_t >= 0 && !mbar_wait(bar(C::kBarSFree + prev_t), static_cast<uint32_t>(prev_l) & 1, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t qbase = base + C::kQOff + t * C::kTileBytes;
+  #pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              // 16 elements (32 bytes) per step inside a 64-wide swizzle column
+              const uint32_t o = (kk >> 2) * C::kSubBytes + (kk & 3) * 32;
+              mma_f16_ss(tmem + C::kColS, sdesc_sw128(qbase + o, 16, 1024), sdesc_sw128(kbase + o, 16, 1024), idesc_qk,
+                         kk > 0 ? 1u : 0u);
+            }
+            mma_commit(bar(C::kBarSFull + t));
+            qk_issued[t] = lt + 1;  // lets the PV issuer queue behind this QK
+            prev_t = t;
+            prev_l = lt;
           }
-          mma_commit(bar(C::kBarSFull + t));
-          qk_issued[t] = lt + 1;  // lets the PV issuer queue behind this QK
-          prev_t = t;
-          prev_l = lt;
+          if (!ok) break;
+          mma_commit(bar(C::kBarKEmpty + s));  // every QK of K_j retired
         }
-        if (!ok) break;
-        mma_commit(bar(C::kBarKEmpty + s));  // every QK of K_j retired
+        // every MMA issued above has retired before TMEM can be released
+        mma_commit(bar(C::kBarDrain));
+        mbar_wait_drain(bar(C::kBarDrain), 0);
       }
-      // every MMA issued above has retired before TMEM can be released
-      mma_commit(bar(C::kBarDrain));
-      mbar_wait_drain(bar(C::kBarDrain), 0);
-    }
-  } else if (warp == C::kWarpPV) {
-    // ---------------------------------------------------------------- PV issuer
-    if (lane == 0 && nj > 0) {
-      constexpr uint32_t idesc_pv = idesc_bf16(128, 128, true);
-      bool ok = true;
-      for (int jj = 0; ok && jj < nj; ++jj) {
-        const int j = ub + jj;
-        const int s = jj % C::kVStages;
-        const uint32_t vbase = base + C::kVOff + s * C::kTileBytes;
-        bool v_ready = false;
-#pragma unroll
-        for (int t = 0; t < 2; ++t) {
-          const int kb = t ? kb1 : kb0, ke = t ? ke1 : ke0;
-          if (!ok || j < kb || j >= ke) continue;
-          const int lt = j - kb;
-          const int nt = ke - kb;
-          // QK_t(lt+1) is on the softmax's critical path and this P·V is not (its P buffer is
-          // reused only a block later): let that QK reach the tensor core first (bounded;
-          // the order never affects results)
-          if (lt + 1 < nt) {
-            for (int spin = 0; spin < 4096 && qk_issued[t] < lt + 2 && !*abort_flag; ++spin) __nanosleep(32);
+    } else if (warp == C::kWarpPV) {
+      // ---------------------------------------------------------------- PV issuer
+      if (lane == 0 && nj > 0) {
+        constexpr uint32_t idesc_pv = idesc_bf16(128, 128, true);
+        bool ok = true;
+        for (int jj = 0; ok && jj < nj; ++jj) {
+          const int j = ub + jj;
+          const int s = jj % C::kVStages;
+          const uint32_t vbase = base + C::kVOff + s * C::kTileBytes;
+          bool v_ready = false;
+  #pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            const int kb = t ? kb1 : kb0, ke = t ? ke1 : ke0;
+            if (!ok || j < kb || j >= ke) continue;
+            const int lt = j - kb;
+            const int nt = ke - kb;
+            // QK_t(lt+1) is on the softmax's critical path and this P·V is not (its P buffer is
+            // reused only a block later): let that QK reach the tensor core first (bounded;
+            // the order never affects results)
+            if (lt + 1 < nt) {
+              for (int spin = 0; spin < 4096 && qk_issued[t] < lt + 2 && !*abort_flag; ++spin) __nanosleep(32);
+            }
+            if (!mbar_wait(bar(C::kBarPFull + t), static_cast<uint32_t>(lt) & 1, abort_flag) ||
+                (!v_ready &&
+                 !mbar_wait(bar(C::kBarVFull + s), static_cast<uint32_t>(jj / C::kVStages) & 1, abort_flag))) {
+              ok = false;
+              break;
+            }
+            v_ready = true;
+            tc_fence_after();
+            const uint32_t pcol = tmem + C::kColP + 64 * t;
+            const uint32_t ocol = tmem + (t ? C::kColO1 : C::kColO0);
+  #pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              // B = V tile, MN-major: 16 key rows per step (2048 B), D-halves one swizzle column apart
+              mma_f16_ts(ocol, pcol + kk * 8, sdesc_sw128(vbase + kk * 2048, C::kSubBytes, 1024), idesc_pv,
+                         (lt > 0 || kk > 0) ? 1u : 0u);
+            }
+            mma_commit(bar(C::kBarPVDone + t));
+            if (lt == nt - 1) mma_commit(bar(C::kBarOFinal + t));
           }
-          if (!mbar_wait(bar(C::kBarPFull + t), static_cast<uint32_t>(lt) & 1, abort_flag) ||
-              (!v_ready && !mbar_wait(bar(C::kBarVFull + s), static_cast<uint32_t>(jj / C::kVStages) & 1, abort_flag))) {
-            ok = false;
-            break;
-          }
-          v_ready = true;
-          tc_fence_after();
-          const uint32_t pcol = tmem + C::kColP + 64 * t;
-          const uint32_t ocol = tmem + (t ? C::kColO1 : C::kColO0);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            // B = V tile, MN-major: 16 key rows per step (2048 B), D-halves one swizzle column apart
-            mma_f16_ts(ocol, pcol + kk * 8, sdesc_sw128(vbase + kk * 2048, C::kSubBytes, 1024), idesc_pv,
-                       (lt > 0 || kk > 0) ? 1u : 0u);
-          }
-          mma_commit(bar(C::kBarPVDone + t));
-          if (lt == nt - 1) mma_commit(bar(C::kBarOFinal + t));
+          // (the two ranges overlap or abut, so some tile needs every key tile of the union;
+          // should none, the copy must still land before its stage is handed back)
+          if (ok && !v_ready)
+            ok = mbar_wait(bar(C::kBarVFull + s), static_cast<uint32_t>(jj / C::kVStages) & 1, abort_flag);
+          if (!ok) break;
+          mma_commit(bar(C::kBarVEmpty + s));  // every P·V of V_j retired
         }
-        // (the two ranges overlap or abut, so some tile needs every key tile of the union;
-        // should none, the copy must still land before its stage is handed back)
-        if (ok && !v_ready)
-          ok = mbar_wait(bar(C::kBarVFull + s), static_cast<uint32_t>(jj / C::kVStages) & 1, abort_flag);
-        if (!ok) break;
-        mma_commit(bar(C::kBarVEmpty + s));  // every P·V of V_j retired
+        mma_commit(bar(C::kBarDrain + 1));
+        mbar_wait_drain(bar(C::kBarDrain + 1), 0);
       }
-      mma_commit(bar(C::kBarDrain + 1));
-      mbar_wait_drain(bar(C::kBarDrain + 1), 0);
     }
-  }
   } else {
     regs_inc<PairMaskedCfg::kRegSoftmax>();
     // ---------------------------------------------------------------- softmax warps
