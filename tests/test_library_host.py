@@ -86,6 +86,11 @@ def _attn(**over):
     (dict(layout=2), 1),
     (dict(cq=ctypes.c_void_p(0x10000)), 1),
     (dict(B=0), 1),
+    (dict(mask=ctypes.c_void_p(0x10000)), 1),                             # a mask without its shape
+    (dict(mask=ctypes.c_void_p(0x10000), mshape=5), 1),                   # unknown mask shape
+    (dict(pse=ctypes.c_void_p(0x10008)), 1),                              # pse not 16-byte aligned
+    (dict(layout=2, mask=ctypes.c_void_p(0x10000), mshape=1), 2),         # atten_mask with TND
+    (dict(layout=2, pse=ctypes.c_void_p(0x10000)), 2),                    # pse with TND
 ])
 def test_attn_fwd_rejects_before_launch(over, status):
     st, msg = _attn(**over)
